@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the routed MoE FFN layer: MoE-layer tokens/s on B200.
+
+Default workload: the decode layer (d_model 4096, d_ff 2048, 256 MXFP4 routed
+experts, top-8 softmax routing, bf16 activations, one bf16 shared expert of
+d_ff 2048) at T = 8 tokens. One step = one moe_layer call (route -> permute ->
+expert FFN + shared expert -> combine) on one batch; batches rotate over 8
+seeded inputs and L2 is flushed (256 MB write) between steps, outside the
+timed events. Other configurations are measured in the same run and reported
+under "breakdown".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs an independent replica on its own
+batches (the path partitions by token batch; no data-path collective) and the
+job value is the sum over ranks of tokens over the slowest rank's time.
+--impl reference times the oracle (plain C, host cores) on the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec (decode T<=8, prefill T=4096); % HBM / FP4-TC roofline"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+NBATCH = 8
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ---- device setup (product path only: no oracle here) -------------------------
+
+class DeviceLayer:
+    """Weights of one layer config on the device, built with the library's own
+    quantiser and packer from the seeded generator's fp32 normals."""
+
+    def __init__(self, M, torch, cfg, seed=0):
+        self.M, self.torch, self.cfg = M, torch, cfg
+        dev = torch.device("cuda")
+        self.dims = self.dims_for(cfg.T)
+        self.packed = {}
+        chunk = 16
+        for tid, which in ((synth.W1, M.MOE_MAT_W1), (synth.W3, M.MOE_MAT_W3), (synth.W2, M.MOE_MAT_W2)):
+            N, K = (cfg.F, cfg.d) if tid != synth.W2 else (cfg.d, cfg.F)
+            q2k = cfg.wfmt == "q2k"
+            per_e_a = N * K // 256 * 84 if q2k else N * K // 2
+            per_e_b = 0 if q2k else N * K // 32
+            canon = torch.empty(cfg.E * (per_e_a + per_e_b), dtype=torch.uint8, device=dev)
+            f32 = torch.empty(chunk * N * K, dtype=torch.float32, device=dev)
+            tmp = torch.empty(chunk * (per_e_a + per_e_b), dtype=torch.uint8, device=dev)
+            for e0 in range(0, cfg.E, chunk):
+                ne = min(chunk, cfg.E - e0)
+                for j in range(ne):
+                    synth.normal_f32_device(seed, tid, e0 + j, N * K, 0.0, cfg.w_std, out=f32[j * N * K:(j + 1) * N * K])
+                cd = M.make_dims(1, cfg.d, cfg.F, ne, 1, wfmt=self.dims.wfmt)
+                M.moe_quantize_weights(cd, which, f32, tmp)
+                canon[e0 * per_e_a:(e0 + ne) * per_e_a].copy_(tmp[:ne * per_e_a])
+                if per_e_b:
+                    base = cfg.E * per_e_a
+                    canon[base + e0 * per_e_b: base + (e0 + ne) * per_e_b].copy_(
+                        tmp[ne * per_e_a: ne * (per_e_a + per_e_b)])
+            out = torch.empty(M.moe_packed_size(self.dims, which), dtype=torch.uint8, device=dev)
+            M.moe_pack_weights(self.dims, which, canon, out)
+            self.packed[which] = out
+            del canon, f32, tmp
+        to16 = lambda a: torch.from_numpy(a.astype(np.int16)).to(dev)
+        self.wr = to16(synth.make_router(cfg, seed)) if cfg.has_router else None
+        b = synth.make_bias(cfg, seed)
+        self.bias = torch.from_numpy(b).to(dev) if b is not None else None
+        sh = synth.shared_weights_bf16(cfg, seed)
+        self.sh = [to16(a) for a in sh] if sh is not None else [None] * 3
+        self.weights = M.make_weights(self.packed[M.MOE_MAT_W1], self.packed[M.MOE_MAT_W3],
+                                      self.packed[M.MOE_MAT_W2], *self.sh, self.wr, self.bias)
+        torch.cuda.synchronize()
+
+    def dims_for(self, T):
+        M, cfg = self.M, self.cfg
+        return M.make_dims(T, cfg.d, cfg.F, cfg.E, cfg.k,
+                           M.MOE_ROUTE_HASH if cfg.route == "hash" else M.MOE_ROUTE_SOFTMAX_TOPK,
+                           M.MOE_A_MXFP8 if cfg.act == "mxfp8" else M.MOE_A_BF16,
+                           M.MOE_W_Q2K if cfg.wfmt == "q2k" else M.MOE_W_MXFP4,
+                           cfg.Fs if cfg.Fs else 0)
+
+    def with_weights(self, cfg):
+        """The same routed experts under another config of equal dims and format."""
+        other = object.__new__(DeviceLayer)
+        other.__dict__.update(self.__dict__)
+        other.cfg = cfg
+        other.dims = other.dims_for(cfg.T)
+        M, torch = self.M, self.torch
+        dev = torch.device("cuda")
+        to16 = lambda a: torch.from_numpy(a.astype(np.int16)).to(dev)
+        other.wr = to16(synth.make_router(cfg)) if cfg.has_router else None
+        b = synth.make_bias(cfg)
+        other.bias = torch.from_numpy(b).to(dev) if b is not None else None
+        other.sh = self.sh if cfg.Fs else [None] * 3
+        other.weights = M.make_weights(self.packed[M.MOE_MAT_W1], self.packed[M.MOE_MAT_W3],
+                                       self.packed[M.MOE_MAT_W2], *other.sh, other.wr, other.bias)
+        return other
+
+
+def touched_experts(M, torch, layer, x_d, tok_d, T):
+    dims = layer.dims_for(T)
+    ws = torch.empty(M.moe_workspace_size(dims), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((T, layer.cfg.k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, layer.cfg.k), dtype=torch.float32, device="cuda")
+    M.moe_route(dims, x_d, layer.weights, tok_d, idx, w, ws)
+    return idx.cpu().numpy()
+
+
+def algorithmic_ffn_bytes(cfg, n_experts_touched):
+    """Routed-expert weight bytes one layer call must read (codes + scales the
+    decode kernels use), counted once per touched expert."""
+    if cfg.wfmt == "q2k":
+        per = 3 * cfg.F * cfg.d // 256 * 84
+    else:
+        per = 3 * (cfg.F * cfg.d // 2 + cfg.F * cfg.d // 32)
+    return per * n_experts_touched
+
+
+def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=False):
+    """Times `steps` moe_layer calls; returns a dict of per-step times (ms)."""
+    cfg = layer.cfg
+    dev = torch.device("cuda")
+    dims = layer.dims_for(T)
+    ws = torch.empty(M.moe_workspace_size(dims), dtype=torch.uint8, device=dev)
+    xs, toks = [], []
+    for b in range(batches):
+        c = cfg.with_T(T)
+        xs.append(torch.from_numpy(synth.make_x(c, 0, 1000 * rank + b).astype(np.int16)).to(dev))
+        toks.append(torch.from_numpy(synth.make_token_ids(c, 0, 1000 * rank + b)).to(dev)
+                    if cfg.route == "hash" else None)
+    y = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    if e2e:
+        xh = [torch.empty((T, cfg.d), dtype=torch.int16).pin_memory() for _ in range(batches)]
+        for b in range(batches):
+            xh[b].copy_(xs[b].cpu())
+        th = [t.cpu().pin_memory() if t is not None else None for t in toks]
+        yh = torch.empty((T, cfg.d), dtype=torch.float32).pin_memory()
+        xd = torch.empty((T, cfg.d), dtype=torch.int16, device=dev)
+        td = torch.empty(T, dtype=torch.int32, device=dev) if cfg.route == "hash" else None
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+
+    def step(i, timed):
+        b = i % batches
+        flush.fill_(i & 0xFF)
+        if timed:
+            ev[i][0].record(stream)
+            if not e2e:
+                M.moe_debug_set_ffn_events(fev[i][0], fev[i][1])
+        if e2e:
+            xd.copy_(xh[b], non_blocking=True)
+            if td is not None:
+                td.copy_(th[b], non_blocking=True)
+            M.moe_layer(dims, layer.weights, xd, td, y, ws)
+            yh.copy_(y, non_blocking=True)
+        else:
+            M.moe_layer(dims, layer.weights, xs[b], toks[b], y, ws)
+        if timed:
+            if not e2e:
+                M.moe_debug_set_ffn_events(None, None)
+            ev[i][1].record(stream)
+
+    for i in range(warmup):
+        step(i, False)
+    barrier(torch, world)
+    torch.cuda.synchronize()
+    n0 = M.moe_debug_launch_count()
+    for i in range(steps):
+        step(i, True)
+    torch.cuda.synchronize()
+    n1 = M.moe_debug_launch_count()
+    barrier(torch, world)
+    if M.moe_get_device_error() != 0:
+        raise RuntimeError("device error word set during the benchmark")
+    times = [a.elapsed_time(b) for a, b in ev]
+    out = {"ms": times, "launches": n1 - n0}
+    if not e2e:
+        out["ffn_ms"] = [a.elapsed_time(b) for a, b in fev]
+    return out
+
+
+def barrier(torch, world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(torch, world, v):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self):
+        self.proc, self.path = None, None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+            dev = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0]
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", dev, f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                try:
+                    rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
+                except ValueError:
+                    pass
+        os.remove(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[3]) if v.lower() == "active"})
+        loaded = [r[0] for r in rows if r[2] > 150.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---- CPU baseline: the oracle on the host cores ---------------------------------
+
+def oracle_sample(cfg, T, n_tokens, min_seconds, seed=0, batch=0):
+    """Times the oracle's layer on the first n_tokens of a batch; returns
+    (tokens/s, threads, seconds, description)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from harness import host_weights
+    c = cfg.with_T(T)
+    x = synth.make_x(c, seed, batch)
+    tok = synth.make_token_ids(c, seed, batch) if c.route == "hash" else None
+    wr = synth.make_router(c, seed) if c.has_router else None
+    bias = synth.make_bias(c, seed)
+    sh = synth.shared_weights_bf16(c, seed)
+    toks = np.arange(n_tokens, dtype=np.int32)
+    if c.route == "hash":
+        idx, _, _ = oracle.hash_route(tok[:n_tokens], c.E, c.k)
+    else:
+        idx, _ = oracle.topk_softmax(oracle.router_logits(x[:n_tokens], wr, bias), c.k)
+    hw = host_weights(c, seed)
+    hw.ensure(np.unique(idx))
+    ow = hw.oracle_layer(c, wr, bias, sh)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.layer_tokens(ow, x, toks, tok)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= 20:
+            break
+    return reps * n_tokens / el, oracle.num_threads(), el, \
+        f"{reps} x oracle layer on {n_tokens} token(s) of the {cfg.name} T={T} batch"
+
+
+# ---- main -------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--T", type=int, default=8)
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    cfg = synth.CONFIGS["decode"].with_T(args.T)
+    workload = (f"decode layer T={args.T}: d_model 4096, d_ff 2048, 256 MXFP4 routed experts, top-8 softmax "
+                f"routing, bf16 activations, bf16 shared expert d_ff 2048")
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per_step = []
+        for i in range(args.warmup + args.steps):
+            tps, threads, el, desc = oracle_sample(cfg, args.T, args.T, 0.0, batch=i % NBATCH)
+            if i >= args.warmup:
+                per_step.append(args.T / tps)
+        ms = 1000 * statistics.mean(per_step)
+        val = args.T / (ms / 1000)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload, "T": args.T},
+            "cpu_baseline": {"kind": "oracle", "value": val, "unit": UNIT, "cores": threads,
+                             "sample": f"each step: oracle layer on the {args.T} tokens of one batch"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    import routed_expert_ffn_05_b200 as M
+
+    t0 = time.time()
+    base = DeviceLayer(M, torch, synth.CONFIGS["decode"])
+    log(f"[bench] MXFP4 layer built in {time.time() - t0:.1f}s")
+    layer = base.with_weights(cfg)
+
+    clocks = Clocks()
+    clocks.start()
+    r = measure(M, torch, layer, args.T, args.steps, args.warmup, rank, world)
+    ck = clocks.stop()
+    total_s = max_over_ranks(torch, world, sum(r["ms"]) / 1000.0)
+    value = world * args.T * args.steps / total_s
+    ms_per_step = 1000.0 * total_s / args.steps
+
+    e = measure(M, torch, layer, args.T, args.steps, args.warmup, rank, world, e2e=True)
+    e2e_s = max_over_ranks(torch, world, sum(e["ms"]) / 1000.0)
+
+    # roofline of the routed-expert FFN (the dominant stage), per step
+    hbm, bf16, src = peaks()
+    xb = torch.from_numpy(synth.make_x(cfg, 0, 1000 * rank).astype(np.int16)).cuda()
+    idx = touched_experts(M, torch, layer, xb, None, args.T)
+    U = len(np.unique(idx))
+    ffn_ms = statistics.mean(r["ffn_ms"][::NBATCH]) if r["ffn_ms"] else float("nan")
+    alg = algorithmic_ffn_bytes(cfg, U)
+    achieved = alg / (ffn_ms / 1000.0) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "mxfp4 x bf16 -> fp32", "data": "synthetic",
+        "config": {"workload": workload, "T": args.T, "batches": NBATCH,
+                   "l2": "flushed between steps (256 MB write), flush outside the timed events",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"kernel": "routed expert FFN (gate/up + down)", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_source": src, "traffic": None,
+                     "algorithmic_bytes": alg, "experts_touched": U, "ffn_ms": ffn_ms},
+        "e2e": {"value": world * args.T * args.steps / e2e_s, "unit": UNIT,
+                "h2d_bytes_per_step": args.T * cfg.d * 2, "d2h_bytes_per_step": args.T * cfg.d * 4},
+        "gpu_launches": r["launches"], "gpu_launches_per_step": r["launches"] / args.steps,
+        "clocks": ck,
+    }
+
+    if not args.no_breakdown and rank == 0:
+        bd = {}
+        for T in (1, 2, 4, 8):
+            rr = measure(M, torch, base.with_weights(synth.CONFIGS["decode"].with_T(T)), T, 20, 3, rank, 1)
+            bd[f"decode_T{T}"] = {"tokens_per_s": T / (statistics.mean(rr["ms"]) / 1000),
+                                  "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
+        for name in ("prefill", "hash"):
+            c = synth.CONFIGS[name]
+            rr = measure(M, torch, base.with_weights(c), c.T, 3, 3, rank, 1, batches=2)
+            bd[name] = {"T": c.T, "tokens_per_s": c.T / (statistics.mean(rr["ms"]) / 1000),
+                        "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
+        line["breakdown"] = bd
+
+    if not args.no_cpu and world == 1 and rank == 0:
+        tps, threads, el, desc = oracle_sample(cfg, args.T, args.T, 10.0)
+        line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": desc, "seconds": el}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+/*
+ * moe.h — C ABI of the routed mixture-of-experts FFN layer over block-quantised
+ * expert weights (libmoe.so, CUDA, sm_100a).
+ *
+ * The layer is the sparse MoE FFN of DeepSeek V4 Flash as the DwarfStar 4
+ * pages describe it:
+ *  - routed experts are quantised while the shared experts, projections and
+ *    router stay unquantised ("DS4", dibi8.com, "Key architectural
+ *    innovations" item 1; "DwarfStar", hysenlabs.com, "Model support and
+ *    quantisation");
+ *  - routed-expert weights are MXFP4 (the released FP4 weights kept as-is) or
+ *    a 2-bit Q2_K-style format (hysenlabs.com, same section);
+ *  - experts are picked by hashing or by a router ("DeepSeek V4 Flash ... on a
+ *    Mac", grapeot.me, opening section: "hash MoE routing");
+ *  - expert work is batched onto FP4 matrix instructions on Blackwell
+ *    (hysenlabs.com, "Model support and quantisation").
+ * Each expert is a SwiGLU FFN: h = silu(W1 a) * (W3 a), o = W2 h, with W1, W3
+ * of shape [d_ff][d_model] and W2 of shape [d_model][d_ff]; quantisation
+ * blocks run along the input dimension. The layer output is
+ *     y[t] = sum_{j=0..k-1} w[t,j] * o_{e(t,j)}(x[t])  (+ shared expert (x[t])).
+ *
+ * Conventions for every entry point:
+ *  - Pointers are DEVICE pointers unless stated otherwise; the caller owns and
+ *    allocates every buffer. Scratch comes from the caller's workspace `ws`
+ *    (size from moe_workspace_size, 256-byte aligned); the library allocates
+ *    no device memory and keeps no per-call state.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream). Arguments are checked on the host first: a bad argument returns
+ *    MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED and launches nothing.
+ *  - Errors found by a kernel (an expert index outside [0, E), hash routing
+ *    that needs more than 1024 draws for one token, a bounded wait that gave
+ *    up) set a per-device error word; the outputs of that call are then
+ *    undefined. Read and clear it with moe_get_device_error.
+ *  - bf16 values travel as uint16_t bit patterns. Row-major everywhere.
+ *  - Calls on distinct workspaces may run concurrently; weights are read-only.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size or shape, misaligned pointer */
+    MOE_ERR_UNSUPPORTED = 2, /* a valid combination this build does not implement */
+    MOE_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, copy, attribute) */
+    MOE_ERR_DEVICE = 4,      /* the device error word was set (moe_get_device_error) */
+    MOE_ERR_TIMEOUT = 5      /* a bounded device wait gave up */
+} moe_status;
+
+/* Routed-expert weight format. */
+typedef enum { MOE_W_MXFP4 = 1, MOE_W_Q2K = 2 } moe_wfmt;
+/* Activation mode of the routed experts: bf16 ("w4a16") or MXFP8 E4M3 with
+ * per-32 E8M0 scales ("w4a8"; x and the hidden h are both quantised). */
+typedef enum { MOE_A_BF16 = 0, MOE_A_MXFP8 = 1 } moe_amode;
+/* Routing: top-k of bf16 router logits with softmax gates, or hash routing. */
+typedef enum { MOE_ROUTE_SOFTMAX_TOPK = 0, MOE_ROUTE_HASH = 1 } moe_rmode;
+
+/* Device error codes (moe_get_device_error). */
+enum { MOE_DEVERR_NONE = 0, MOE_DEVERR_EXPERT_RANGE = 1, MOE_DEVERR_HASH_CAP = 2,
+       MOE_DEVERR_TIMEOUT = 3 };
+
+/* Layer shape. Limits: d_model and d_ff multiples of 256 (of 32 for MXFP4),
+ * 1 <= k <= min(E, 32), E <= 1024, T*k < 2^31. */
+typedef struct {
+    int32_t T;            /* tokens in this call (>= 0) */
+    int32_t d_model;      /* d */
+    int32_t d_ff;         /* F, routed expert hidden size */
+    int32_t E;            /* routed experts */
+    int32_t k;            /* experts per token */
+    int32_t route;        /* moe_rmode */
+    int32_t act;          /* moe_amode */
+    int32_t wfmt;         /* moe_wfmt */
+    int32_t d_ff_shared;  /* shared expert hidden size, 0 = no shared expert */
+} moe_dims;
+
+/* Weights of one layer (device pointers, read-only).
+ *  w1, w3, w2: routed experts in the PACKED device layout written by
+ *              moe_pack_weights (size from moe_packed_size);
+ *  sw1, sw3:   shared expert bf16 [d_ff_shared][d_model], sw2 bf16
+ *              [d_model][d_ff_shared], plain row-major; NULL when there is none;
+ *  w_router:   router bf16 [E][d_model] (NULL for hash routing);
+ *  router_bias: fp32 [E] added to the logits, or NULL. */
+typedef struct {
+    const void *w1, *w3, *w2;
+    const uint16_t *sw1, *sw3, *sw2;
+    const uint16_t *w_router;
+    const float *router_bias;
+} moe_weights;
+
+/* Which routed-expert matrix: gate W1, up W3 ([E][d_ff][d_model]) or down W2
+ * ([E][d_model][d_ff]). */
+enum { MOE_MAT_W1 = 1, MOE_MAT_W3 = 3, MOE_MAT_W2 = 2 };
+
+MOE_API const char *moe_status_string(moe_status s);
+
+/* Bytes of workspace that moe_route .. moe_layer need for these dims (all
+ * entry points share one workspace layout). Host only. */
+MOE_API moe_status moe_workspace_size(const moe_dims *dims, size_t *bytes);
+
+/* ---- weights ------------------------------------------------------------
+ * CANONICAL layout of one routed-expert matrix with N rows and K = input dim
+ * (N = d_ff, K = d_model for W1/W3; N = d_model, K = d_ff for W2):
+ *   MXFP4: codes u8 [E][N][K/2] (element 2i in the low nibble, OCP E2M1)
+ *          followed by scales u8 [E][N][K/32] (E8M0) — E*N*K*17/32 bytes;
+ *   Q2_K:  [E][N][K/256] super-blocks of 84 bytes: 16 bytes sc|m<<4,
+ *          64 bytes of 2-bit quants (quant n at byte n/4, bits 2*(n%4)),
+ *          fp16 d, fp16 dmin; w = d*sc*q - dmin*m.
+ */
+
+/* Quantise fp32 weights [E][N][K] (device) into the canonical layout
+ * (device). MXFP4: per 32-block scale 2^(floor(log2 amax) - 2), elements
+ * rounded to nearest-even E2M1 with saturation, all-zero block -> scale 127.
+ * Q2_K: the min-max rule documented with the format. One-time, offline. */
+MOE_API moe_status moe_quantize_weights(const moe_dims *dims, int32_t which, const float *w,
+                                void *canonical, void *stream);
+
+/* Device bytes of one packed matrix (host only). */
+MOE_API moe_status moe_packed_size(const moe_dims *dims, int32_t which, size_t *bytes);
+
+/* Re-lay one canonical matrix (device) into the packed device layout used by
+ * the kernels (device). One-time. `canonical` and `packed` must not overlap;
+ * both 256-byte aligned. */
+MOE_API moe_status moe_pack_weights(const moe_dims *dims, int32_t which, const void *canonical,
+                            void *packed, void *stream);
+
+/* ---- the layer, stage by stage ---------------------------------------------
+ * Router logits are fp32 in one fixed order (32 contiguous chunks of d/32,
+ * each a running fma from +0, then a balanced tree of adjacent pairs, then
+ * the bias), so that expert choice is deterministic and reproducible.
+ * topk_idx int32 [T][k], topk_w fp32 [T][k]; ties go to the lower expert index,
+ * NaN logits last; gates are the softmax of the k chosen logits. Hash routing
+ * (token_ids int32 [T], required): SplitMix64 seeded with the token id, expert =
+ * output mod E, repeats skipped, gates 1/k. */
+MOE_API moe_status moe_route(const moe_dims *dims, const uint16_t *x, const moe_weights *weights,
+                     const int32_t *token_ids, int32_t *topk_idx, float *topk_w, void *ws,
+                     void *stream);
+
+/* Token-by-expert histogram, exclusive scan and stable permutation:
+ * counts int32 [E], offsets int32 [E+1], perm int32 [T*k] (row -> slot t*k+j,
+ * rows of one expert in ascending slot order), inv_perm int32 [T*k]
+ * (slot -> row). Bit-exact and deterministic. */
+MOE_API moe_status moe_permute(const moe_dims *dims, const int32_t *topk_idx, int32_t *counts,
+                       int32_t *offsets, int32_t *perm, int32_t *inv_perm, void *ws, void *stream);
+
+/* Routed expert FFNs for every permuted row: out_rows fp32 [T*k][d_model],
+ * row r = o_{e}(x[perm[r] / k]) for the expert e whose segment holds r.
+ * x bf16 [T][d_model]. In MXFP8 mode x and h are quantised on the fly. */
+MOE_API moe_status moe_expert_ffn(const moe_dims *dims, const moe_weights *weights, const uint16_t *x,
+                          const int32_t *offsets, const int32_t *perm, float *out_rows, void *ws,
+                          void *stream);
+
+/* Shared expert: s fp32 [T][d_model] = W2s (bf16(silu(W1s x) * (W3s x))),
+ * bf16 weights and activations, fp32 accumulation. */
+MOE_API moe_status moe_shared_ffn(const moe_dims *dims, const moe_weights *weights, const uint16_t *x,
+                          float *shared_out, void *ws, void *stream);
+
+/* Gate-weighted combine: y fp32 [T][d_model] =
+ * sum_{j ascending} topk_w[t][j] * out_rows[inv_perm[t*k+j]] (+ shared_out[t]).
+ * shared_out may be NULL. */
+MOE_API moe_status moe_combine(const moe_dims *dims, const float *out_rows, const int32_t *inv_perm,
+                       const float *topk_w, const float *shared_out, float *y, void *stream);
+
+/* The whole layer: route -> permute -> expert FFN (+ shared expert) ->
+ * combine, y fp32 [T][d_model]. token_ids is required for hash routing and
+ * ignored otherwise. */
+MOE_API moe_status moe_layer(const moe_dims *dims, const moe_weights *weights, const uint16_t *x,
+                     const int32_t *token_ids, float *y, void *ws, void *stream);
+
+/* Synchronises `stream`, returns the per-device error word in *code (host
+ * pointer) and clears it. Returns MOE_ERR_DEVICE when it was set. */
+MOE_API moe_status moe_get_device_error(void *stream, int32_t *code);
+
+/* ---- test hooks ------------------------------------------------------------ */
+
+/* Dequantise one matrix of one expert from the PACKED layout: out fp32 [N][K]
+ * (device). Bit-exact decode of the format. */
+MOE_API moe_status moe_debug_dequant(const moe_dims *dims, int32_t which, const void *packed,
+                             int32_t expert, float *out, void *stream);
+
+/* MXFP8-quantise bf16 rows: codes u8 [rows][K], scales u8 [rows][K/32]
+ * (device), the same rule the layer applies to x. */
+MOE_API moe_status moe_debug_quant_act(const uint16_t *x, int32_t rows, int32_t K, uint8_t *codes,
+                               uint8_t *scales, void *stream);
+
+/* Number of kernels this library has launched in this process (host counter,
+ * all devices and threads). For benchmarks that report their launch count. */
+MOE_API uint64_t moe_debug_launch_count(void);
+
+/* Profiling hook: when both are non-NULL, moe_layer and moe_expert_ffn record
+ * `before` (a cudaEvent_t) on their stream right before the first routed-expert
+ * FFN kernel and `after` right after the last one. NULL, NULL turns it off.
+ * Process-wide; not for concurrent use from several threads. */
+MOE_API moe_status moe_debug_set_ffn_events(void *before, void *after);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

@@ -1,0 +1,44 @@
+// Gate-weighted combine: y[t] = sum_{j ascending} w[t,j] * o[inv_perm[t*k+j]]
+// (+ shared expert s[t]), fp32, the k terms in a fixed order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ out_rows,
+                                                      const int32_t *__restrict__ inv_perm,
+                                                      const float *__restrict__ gates,
+                                                      const float *__restrict__ shared, int d, int k,
+                                                      float *__restrict__ y) {
+    const int t = blockIdx.y;
+    const int i4 = blockIdx.x * blockDim.x + threadIdx.x;  // float4 index
+    if (i4 * 4 >= d) return;
+    float4 acc = shared ? reinterpret_cast<const float4 *>(shared + (int64_t)t * d)[i4]
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+        const int64_t s = (int64_t)t * k + j;
+        const float g = gates[s];
+        const float4 o = reinterpret_cast<const float4 *>(out_rows + (int64_t)inv_perm[s] * d)[i4];
+        sum.x = fmaf(g, o.x, sum.x);
+        sum.y = fmaf(g, o.y, sum.y);
+        sum.z = fmaf(g, o.z, sum.z);
+        sum.w = fmaf(g, o.w, sum.w);
+    }
+    acc.x += sum.x;
+    acc.y += sum.y;
+    acc.z += sum.z;
+    acc.w += sum.w;
+    reinterpret_cast<float4 *>(y + (int64_t)t * d)[i4] = acc;
+}
+
+cudaError_t launch_combine(const moe_dims &d, const float *out_rows, const int32_t *inv_perm,
+                           const float *gates, const float *shared, float *y, cudaStream_t s) {
+    if (d.T == 0) return cudaSuccess;
+    const dim3 grid(ceil_div(d.d_model / 4, 256), d.T);
+    combine_kernel<<<grid, 256, 0, s>>>(out_rows, inv_perm, gates, shared, d.d_model, d.k, y);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

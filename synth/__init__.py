@@ -33,6 +33,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "synth.c")
 _SO = os.path.join(_HERE, "libsynth.so")
+_GPU_SRC = os.path.join(_HERE, "synth_gpu.cu")
+_GPU_SO = os.path.join(_HERE, "libsynth_gpu.so")
 
 # Tensor ids: each tensor of a workload draws from its own Philox key.
 X, WR, W1, W3, W2, S1, S3, S2, TOK, ZIPF = range(1, 11)
@@ -45,6 +47,11 @@ def build(force: bool = False) -> str:
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
                                "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
         os.replace(tmp, _SO)
+    if force or not os.path.exists(_GPU_SO) or os.path.getmtime(_GPU_SO) < os.path.getmtime(_GPU_SRC):
+        tmp = _GPU_SO + f".tmp{os.getpid()}"
+        subprocess.check_call(["nvcc", "-O3", "-gencode", "arch=compute_100a,code=sm_100a", "-Xcompiler",
+                               "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared", _GPU_SRC, "-o", tmp])
+        os.replace(tmp, _GPU_SO)
     return _SO
 
 
@@ -70,6 +77,31 @@ def _lib():
             getattr(L, f).restype = None
         _lib_handle = L
     return _lib_handle
+
+
+_gpu_handle = None
+
+
+def normal_f32_device(seed, tensor, sub, n, mean=0.0, std=1.0, first=0, out=None, stream=None):
+    """Fill a float32 CUDA tensor with the same normal stream as normal_f32 (device copy of
+    the generator; bench-sized tensors only)."""
+    import torch
+    global _gpu_handle
+    if _gpu_handle is None:
+        build()
+        L = ctypes.CDLL(_GPU_SO)
+        L.synth_gpu_normal_f32.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint64,
+                                           ctypes.c_int64, ctypes.c_double, ctypes.c_double, ctypes.c_void_p,
+                                           ctypes.c_void_p]
+        L.synth_gpu_normal_f32.restype = ctypes.c_int
+        _gpu_handle = L
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    rc = _gpu_handle.synth_gpu_normal_f32(seed, tensor, sub, first, n, mean, std, out.data_ptr(), s)
+    if rc != 0:
+        raise RuntimeError(f"synth_gpu_normal_f32 failed: cuda error {rc}")
+    return out
 
 
 def _ptr(a: np.ndarray) -> int:

@@ -73,12 +73,32 @@ static inline double normal_at(uint64_t seed, uint32_t tensor, uint32_t sub, uin
     return (j & 1) ? rad * sin(ang) : rad * cos(ang);
 }
 
+/* Both normals of Box-Muller pair b (normals 2b and 2b+1). */
+static inline void normal_pair(uint64_t seed, uint32_t tensor, uint32_t sub, uint64_t b, double z[2]) {
+    uint32_t r[4];
+    block(seed, tensor, sub, 0u, b, r);
+    const double u1 = u53(r[0], r[1]);
+    const double u2 = u53(r[2], r[3]);
+    const double rad = sqrt(-2.0 * log(u1));
+    const double ang = 6.283185307179586476925286766559 * u2;
+    z[0] = rad * cos(ang);
+    z[1] = rad * sin(ang);
+}
+
 /* out[i] = (float)(mean + std * z_{first+i}) */
 void synth_normal_f32(uint64_t seed, uint32_t tensor, uint32_t sub, uint64_t first, int64_t n,
                       double mean, double std, float *out) {
+    if (n <= 0) return;
+    const uint64_t b0 = first >> 1, b1 = (first + (uint64_t)n + 1) >> 1;
 #pragma omp parallel for schedule(static)
-    for (int64_t i = 0; i < n; ++i)
-        out[i] = (float)(mean + std * normal_at(seed, tensor, sub, first + (uint64_t)i));
+    for (int64_t b = (int64_t)b0; b < (int64_t)b1; ++b) {
+        double z[2];
+        normal_pair(seed, tensor, sub, (uint64_t)b, z);
+        for (int h = 0; h < 2; ++h) {
+            const int64_t i = 2 * b + h - (int64_t)first;
+            if (i >= 0 && i < n) out[i] = (float)(mean + std * z[h]);
+        }
+    }
 }
 
 /* bfloat16 bit pattern of the float value above, round-to-nearest-even. */

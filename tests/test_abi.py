@@ -1,0 +1,52 @@
+"""The C ABI: the library loads without a GPU, exports every declared entry
+point, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_functions())
+    for n in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer",
+              "moe_workspace_size", "moe_pack_weights", "moe_get_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import routed_expert_ffn_05_b200 as M
+    for n in declared_functions():
+        assert hasattr(M.lib, n), n
+        assert hasattr(M, n) or n == "moe_status_string", n
+
+
+def test_host_side_argument_checks():
+    import routed_expert_ffn_05_b200 as M
+    d = M.make_dims(4, 4096, 2048, 256, 8)
+    assert M.moe_workspace_size(d) > 0
+    assert M.moe_packed_size(d, M.MOE_MAT_W1) >= 256 * 2048 * 4096 * 17 // 32
+    bad = [M.make_dims(4, 4000, 2048, 256, 8), M.make_dims(4, 4096, 2048, 256, 300),
+           M.make_dims(4, 4096, 2048, 4, 8), M.make_dims(-1, 4096, 2048, 256, 8),
+           M.make_dims(4, 4096, 2048, 256, 8, route=7)]
+    for b in bad:
+        with pytest.raises(M.MoeError) as ei:
+            M.moe_workspace_size(b)
+        assert ei.value.status == M.MOE_ERR_INVALID_ARG
+    w = M.make_weights(None, None, None)
+    with pytest.raises(M.MoeError) as ei:  # NULL routed weights: rejected before any launch
+        M.moe_layer(d, w, 0x1000, None, 0x1000, 0x1000, stream=0)
+    assert ei.value.status == M.MOE_ERR_INVALID_ARG
+    with pytest.raises(M.MoeError):        # misaligned workspace
+        M.moe_permute(d, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1001, stream=0)
+    with pytest.raises(M.MoeError):        # hash routing without token ids
+        M.moe_route(M.make_dims(4, 4096, 2048, 256, 8, route=M.MOE_ROUTE_HASH), 0x1000, w, None,
+                    0x1000, 0x1000, 0x1000, stream=0)
+    assert M.status_string(M.MOE_ERR_DEVICE) == "device error word set"
