@@ -169,6 +169,9 @@ def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=
     stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in fev:  # torch creates the CUDA event on first record; the library needs live handles
+        a.record(stream)
+        b.record(stream)
 
     def step(i, timed):
         b = i % batches

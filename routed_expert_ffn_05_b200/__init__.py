@@ -108,7 +108,10 @@ def make_dims(T, d_model, d_ff, E, k, route=MOE_ROUTE_SOFTMAX_TOPK, act=MOE_A_BF
 
 
 def make_weights(w1, w3, w2, sw1=None, sw3=None, sw2=None, w_router=None, router_bias=None) -> moe_weights:
-    return moe_weights(*(_p(a) for a in (w1, w3, w2, sw1, sw3, sw2, w_router, router_bias)))
+    args = (w1, w3, w2, sw1, sw3, sw2, w_router, router_bias)
+    w = moe_weights(*(_p(a) for a in args))
+    w._keep = args  # the struct holds raw pointers: keep the tensors alive with it
+    return w
 
 
 def moe_workspace_size(dims: moe_dims) -> int:
