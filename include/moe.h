@@ -178,6 +178,34 @@ MOE_API moe_status moe_combine(const moe_dims *dims, const float *out_rows, cons
 MOE_API moe_status moe_layer(const moe_dims *dims, const moe_weights *weights, const uint16_t *x,
                      const int32_t *token_ids, float *y, void *ws, void *stream);
 
+/* Size of the scratch array built into the library for moe_layer_static_ws. */
+#define MOE_STATIC_WS_BYTES (16u << 20)
+
+/* moe_layer for callers that cannot allocate device memory. The pages have no
+ * counterpart: this is a deployment convenience of this library.
+ *
+ * Who needs it: programs whose device memory belongs to another allocator (a
+ * serving framework's pool, or an arena fixed at start-up, where one more
+ * cudaMalloc would break the memory budget), latency-critical decode loops
+ * that cannot pay for cudaMalloc / cudaFree (both may synchronise the device
+ * and stall other streams), and deployments that forbid allocation after
+ * initialisation. Instead of a caller workspace it uses one scratch array of
+ * MOE_STATIC_WS_BYTES compiled into the library; every GPU that loads the
+ * library holds that array until the process exits.
+ *
+ * Same arguments, results and errors as moe_layer minus `ws`. Returns
+ * MOE_ERR_INVALID_ARG, launching nothing, when moe_workspace_size(dims) is
+ * larger than MOE_STATIC_WS_BYTES (at d_model 4096, d_ff 2048, E 256, k 8
+ * with a shared expert of d_ff 2048 that holds up to T = 64 tokens). It calls
+ * no cudaMalloc, cudaFree or other allocating routine. The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress, with that
+ * device current); make that first call before any stream capture. All calls
+ * on a device share the one array and it keeps the previous call's contents
+ * (the layer writes every scratch byte before reading it), so calls whose
+ * execution overlaps on the GPU race: serialise them, e.g. on one stream. */
+MOE_API moe_status moe_layer_static_ws(const moe_dims *dims, const moe_weights *weights, const uint16_t *x,
+                                       const int32_t *token_ids, float *y, void *stream);
+
 /* Synchronises `stream`, returns the per-device error word in *code (host
  * pointer) and clears it. Returns MOE_ERR_DEVICE when it was set. */
 MOE_API moe_status moe_get_device_error(void *stream, int32_t *code);

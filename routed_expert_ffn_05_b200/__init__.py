@@ -62,6 +62,7 @@ def _load():
         "moe_get_device_error": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
         "moe_debug_dequant": (ctypes.c_int, [D, i32, vp, i32, vp, vp]),
         "moe_debug_quant_act": (ctypes.c_int, [vp, i32, i32, vp, vp, vp]),
+        "moe_layer_static_ws": (ctypes.c_int, [D, W, vp, vp, vp, vp]),
         "moe_debug_launch_count": (ctypes.c_uint64, []),
         "moe_debug_set_ffn_events": (ctypes.c_int, [vp, vp]),
     }
@@ -164,6 +165,16 @@ def moe_combine(dims, out_rows, inv_perm, topk_w, shared_out, y, stream=None):
 def moe_layer(dims, weights, x, token_ids, y, ws, stream=None):
     _check(lib.moe_layer(ctypes.byref(dims), ctypes.byref(weights), _p(x), _p(token_ids), _p(y), _p(ws),
                          _stream(stream)), "moe_layer")
+
+
+MOE_STATIC_WS_BYTES = 16 << 20
+
+
+def moe_layer_static_ws(dims, weights, x, token_ids, y, stream=None):
+    """moe_layer for callers that cannot allocate device memory: scratch comes from an
+    array built into the library (MOE_STATIC_WS_BYTES per GPU); see include/moe.h."""
+    _check(lib.moe_layer_static_ws(ctypes.byref(dims), ctypes.byref(weights), _p(x), _p(token_ids), _p(y),
+                                   _stream(stream)), "moe_layer_static_ws")
 
 
 def moe_get_device_error(stream=None) -> int:
