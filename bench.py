@@ -135,13 +135,13 @@ def touched_experts(M, torch, layer, x_d, tok_d, T):
 
 
 def algorithmic_ffn_bytes(cfg, n_experts_touched):
-    """Routed-expert weight bytes one layer call must read (codes + scales the
-    decode kernels use), counted once per touched expert."""
+    """Weight bytes one layer call's expert FFN must read: the touched routed
+    experts' codes + scales (once each) and the bf16 shared expert."""
     if cfg.wfmt == "q2k":
         per = 3 * cfg.F * cfg.d // 256 * 84
     else:
         per = 3 * (cfg.F * cfg.d // 2 + cfg.F * cfg.d // 32)
-    return per * n_experts_touched
+    return per * n_experts_touched + 3 * cfg.Fs * cfg.d * 2
 
 
 def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=False):
@@ -310,15 +310,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--T", type=int, default=8)
+    ap.add_argument("--E", type=int, default=256, help="routed experts (smaller only for profiling captures)")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    cfg = synth.CONFIGS["decode"].with_T(args.T)
-    workload = (f"decode layer T={args.T}: d_model 4096, d_ff 2048, 256 MXFP4 routed experts, top-8 softmax "
+    from dataclasses import replace
+    cfg = replace(synth.CONFIGS["decode"].with_T(args.T), E=args.E)
+    workload = (f"decode layer T={args.T}: d_model 4096, d_ff 2048, {args.E} MXFP4 routed experts, top-8 softmax "
                 f"routing, bf16 activations, bf16 shared expert d_ff 2048")
 
     if args.impl == "reference":
@@ -350,7 +353,7 @@ def main():
     import routed_expert_ffn_05_b200 as M
 
     t0 = time.time()
-    base = DeviceLayer(M, torch, synth.CONFIGS["decode"])
+    base = DeviceLayer(M, torch, replace(synth.CONFIGS["decode"], E=args.E))
     log(f"[bench] MXFP4 layer built in {time.time() - t0:.1f}s")
     layer = base.with_weights(cfg)
 
@@ -362,8 +365,11 @@ def main():
     value = world * args.T * args.steps / total_s
     ms_per_step = 1000.0 * total_s / args.steps
 
-    e = measure(M, torch, layer, args.T, args.steps, args.warmup, rank, world, e2e=True)
-    e2e_s = max_over_ranks(torch, world, sum(e["ms"]) / 1000.0)
+    if not args.no_e2e:
+        e = measure(M, torch, layer, args.T, args.steps, args.warmup, rank, world, e2e=True)
+        e2e_s = max_over_ranks(torch, world, sum(e["ms"]) / 1000.0)
+    else:
+        e2e_s = float("nan")
 
     # roofline of the routed-expert FFN (the dominant stage), per step
     hbm, bf16, src = peaks()
@@ -380,7 +386,7 @@ def main():
         "config": {"workload": workload, "T": args.T, "batches": NBATCH,
                    "l2": "flushed between steps (256 MB write), flush outside the timed events",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "roofline": {"kernel": "routed expert FFN (gate/up + down)", "bound": "hbm",
+        "roofline": {"kernel": "expert FFN: routed + shared (gate/up + down kernels)", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_source": src, "traffic": None,
                      "algorithmic_bytes": alg, "experts_touched": U, "ffn_ms": ffn_ms},
@@ -393,11 +399,11 @@ def main():
     if not args.no_breakdown and rank == 0:
         bd = {}
         for T in (1, 2, 4, 8):
-            rr = measure(M, torch, base.with_weights(synth.CONFIGS["decode"].with_T(T)), T, 20, 3, rank, 1)
+            rr = measure(M, torch, base.with_weights(cfg.with_T(T)), T, 20, 3, rank, 1)
             bd[f"decode_T{T}"] = {"tokens_per_s": T / (statistics.mean(rr["ms"]) / 1000),
                                   "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
         for name in ("prefill", "hash"):
-            c = synth.CONFIGS[name]
+            c = replace(synth.CONFIGS[name], E=args.E)
             rr = measure(M, torch, base.with_weights(c), c.T, 3, 3, rank, 1, batches=2)
             bd[name] = {"T": c.T, "tokens_per_s": c.T / (statistics.mean(rr["ms"]) / 1000),
                         "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}

@@ -27,11 +27,11 @@ static cudaEvent_t g_ffn_before = nullptr, g_ffn_after = nullptr;
 
 // Routed-expert FFN bracketed by the optional profiling events.
 static cudaError_t expert_ffn_timed(const moe_dims &d, const moe_weights &w, const uint16_t *x,
-                                    const int32_t *offsets, const int32_t *perm, float *rows, uint8_t *ws,
-                                    const WsLayout &L, cudaStream_t s) {
+                                    const int32_t *offsets, const int32_t *perm, float *rows, float *shared,
+                                    uint8_t *ws, const WsLayout &L, cudaStream_t s, bool prepared = false) {
     cudaError_t e;
     if (g_ffn_before && g_ffn_after && (e = cudaEventRecord(g_ffn_before, s)) != cudaSuccess) return e;
-    if ((e = launch_expert_ffn(d, w, x, offsets, perm, rows, ws, L, s)) != cudaSuccess) return e;
+    if ((e = launch_expert_ffn(d, w, x, offsets, perm, rows, shared, ws, L, s, prepared)) != cudaSuccess) return e;
     if (g_ffn_before && g_ffn_after) return cudaEventRecord(g_ffn_after, s);
     return cudaSuccess;
 }
@@ -172,8 +172,8 @@ moe_status moe_expert_ffn(const moe_dims *dims, const moe_weights *weights, cons
     if (dims->T > 0 && (!x || !offsets || !perm || !out_rows || !aligned(x, 16) || !aligned(out_rows, 16)))
         return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(*dims);
-    return cuda_status(expert_ffn_timed(*dims, *weights, x, offsets, perm, out_rows, static_cast<uint8_t *>(ws),
-                                        L, static_cast<cudaStream_t>(stream)));
+    return cuda_status(expert_ffn_timed(*dims, *weights, x, offsets, perm, out_rows, nullptr,
+                                        static_cast<uint8_t *>(ws), L, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_shared_ffn(const moe_dims *dims, const moe_weights *weights, const uint16_t *x, float *shared_out,
@@ -222,15 +222,19 @@ moe_status moe_layer(const moe_dims *dims, const moe_weights *weights, const uin
     float *rows = reinterpret_cast<float *>(w + L.out_rows);
     float *sh = d.d_ff_shared > 0 ? reinterpret_cast<float *>(w + L.sh_out) : nullptr;
     cudaError_t e;
-    if ((e = launch_route(d, x, *weights, token_ids, idx, gates, reinterpret_cast<float *>(w + L.logits), s)))
-        return cuda_status(e);
-    if ((e = launch_permute(d, idx, counts, offsets, perm, inv, reinterpret_cast<int32_t *>(w + L.blkcnt),
-                            reinterpret_cast<int32_t *>(w + L.blkbase), L.nblk, s)))
-        return cuda_status(e);
-    if (sh && (e = launch_shared_ffn(d, *weights, x, sh, reinterpret_cast<float *>(w + L.sh_h), s)))
-        return cuda_status(e);
-    if ((e = expert_ffn_timed(d, *weights, x, offsets, perm, rows, w, L, s))) return cuda_status(e);
-    return cuda_status(launch_combine(d, rows, inv, gates, sh, y, s));
+    const bool fused = decode_route_applies(d);
+    if (fused) {
+        if ((e = launch_decode_route(d, x, *weights, idx, gates, counts, offsets, perm, inv, w, L, s)))
+            return cuda_status(e);
+    } else {
+        if ((e = launch_route(d, x, *weights, token_ids, idx, gates, reinterpret_cast<float *>(w + L.logits), s)))
+            return cuda_status(e);
+        if ((e = launch_permute(d, idx, counts, offsets, perm, inv, reinterpret_cast<int32_t *>(w + L.blkcnt),
+                                reinterpret_cast<int32_t *>(w + L.blkbase), L.nblk, s)))
+            return cuda_status(e);
+    }
+    if ((e = expert_ffn_timed(d, *weights, x, offsets, perm, rows, sh, w, L, s, fused))) return cuda_status(e);
+    return cuda_status(launch_combine(d, rows, inv, gates, sh, y, s, decode_path_applies(d)));
 }
 
 moe_status moe_get_device_error(void *stream, int32_t *code) {

@@ -2,6 +2,7 @@
 // (+ shared expert s[t]), fp32, the k terms in a fixed order.
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -10,6 +11,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
                                                       const float *__restrict__ gates,
                                                       const float *__restrict__ shared, int d, int k,
                                                       float *__restrict__ y) {
+    grid_dep_wait();  // launched programmatically after the expert FFN: its outputs first
     const int t = blockIdx.y;
     const int i4 = blockIdx.x * blockDim.x + threadIdx.x;  // float4 index
     if (i4 * 4 >= d) return;
@@ -33,12 +35,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 }
 
 cudaError_t launch_combine(const moe_dims &d, const float *out_rows, const int32_t *inv_perm,
-                           const float *gates, const float *shared, float *y, cudaStream_t s) {
+                           const float *gates, const float *shared, float *y, cudaStream_t s, bool pdl) {
     if (d.T == 0) return cudaSuccess;
-    const dim3 grid(ceil_div(d.d_model / 4, 256), d.T);
-    combine_kernel<<<grid, 256, 0, s>>>(out_rows, inv_perm, gates, shared, d.d_model, d.k, y);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ceil_div(d.d_model / 4, 256), d.T);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const int dm = d.d_model, k = d.k;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, out_rows, inv_perm, gates, shared, dm, k, y);
     count_launches(1);
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -1,0 +1,870 @@
+// Decode-sized expert FFN (T <= 8 tokens): one persistent weight-streaming
+// kernel on tensor cores, HBM-bound.
+//
+// Each routed expert is a SwiGLU FFN over MXFP4 weights; the shared expert is
+// bf16 ("DS4", dibi8.com, "Key architectural innovations" item 1; "DwarfStar",
+// hysenlabs.com, "Model support and quantisation"). With at most 8 tokens per
+// expert the layer is a stream over the touched experts' weights, so the
+// kernel is built around keeping HBM busy:
+//  - one CTA per SM with three roles: a producer thread moves weight tiles
+//    HBM -> shared memory with TMA (one 16-32 KB tile per instruction,
+//    128-byte swizzled) through four 34 KB mbarrier stages; eight consumer
+//    warps split K and run mma.sync m16n8k16 (16 weight rows x 8 tokens, fp32
+//    accumulate); an epilogue warp reduces the consumers' partial tiles from a
+//    double buffer and writes the outputs, so consumers never wait for one
+//    another;
+//  - gate/up and down run in the same launch: one work queue holds the shared
+//    expert's gate/up tiles, the routed gate/up tiles, then the down tiles,
+//    largest first; a down tile waits (bounded) on a per-expert count of
+//    finished gate/up tiles;
+//  - MXFP4 codes become f16 with the hardware E2M1 conversion; the E8M0 block
+//    scale is applied per 32-element block in fp32;
+//  - gate/up uses all T tokens as the MMA's N dimension, so its activation
+//    fragments are built once per CTA; outputs for tokens not routed to the
+//    expert are dropped;
+//  - x enters f16 range through an exact per-token power of two; h, rounded to
+//    bf16 as the layer specifies, gets the same treatment per row from its
+//    maximum, recorded with an order-free atomic max;
+//  - launches are chained with programmatic dependent launch, so the shared
+//    expert's gate/up tiles (which need no routing) stream while routing runs;
+//  - every wait is bounded (MOE_DEVERR_TIMEOUT instead of a hang).
+// K is permuted inside each 32-block identically for weights and activations:
+// lane q of a quad holds elements 8q..8q+7 of a block, which cover its MMA
+// k-slots of both k16 steps.
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+#include "tma.h"
+
+namespace moe {
+namespace {
+
+constexpr int kCW = 8;                    // consumer warps
+constexpr int kProducer = kCW;            // warp index of the producer
+constexpr int kEpilogue = kCW + 1;        // warp index of the epilogue warp
+constexpr int kThreads = (kCW + 2) * 32;
+constexpr int kStages = 4;
+constexpr int kStageW = 32768;            // weight tile bytes per stage
+constexpr int kStageS = 2048;             // scale bytes per stage
+constexpr int kMaxE = 1024;
+constexpr int kD = 4096, kF = 2048;       // the dims this tiling is written for
+constexpr int kGuTiles = kF / 16;         // gate/up tiles per routed expert
+constexpr int kDnTiles = kD / 32;         // down tiles (32 rows) per routed expert
+constexpr int kDshTiles = kD / 16;        // shared-expert down tiles
+
+// Work kinds: shared gate/up (bf16, 8 stages of K 512), routed gate/up (MXFP4,
+// 2 stages of K 2048), shared down (bf16, 2 stages of K 1024), routed down
+// (MXFP4, one stage: a 32-row tile over all K).
+enum { kGsh = 0, kGrt = 1, kDsh = 2, kDrt = 3 };
+
+struct DecodeArgs {
+    CUtensorMap m1c, m3c, m2c;  // routed codes, chunked + swizzled
+    CUtensorMap m1s, m3s, m2s;  // routed row-major scales
+    CUtensorMap ms1, ms3, ms2;  // shared expert (bf16), chunked + swizzled
+    int T, E, k, Fs;
+    const int32_t *offsets, *perm;
+    const uint16_t *x;       // [T][d] bf16
+    const float2 *xscale;    // [T] (2^p_t, 2^-p_t): x * 2^-p_t fits f16
+    uint16_t *h;             // routed hidden [S][F] bf16
+    uint32_t *hmax;          // [S] bits of max |h|
+    uint16_t *hs;            // shared hidden [T][Fs] bf16
+    float *out_rows;         // [S][d]
+    float *shared_out;       // [T][d]
+    uint32_t *counters;      // [0] work queue, [1] shared gate/up tiles done, [2+e] expert e tiles done
+    int *err;
+};
+
+struct Smem {
+    uint8_t w[kStages][kStageW];
+    uint8_t s[kStages][kStageS];
+    float red[2][kCW][2][128];   // partial 16x8 tiles per consumer warp
+    uint64_t full[kStages], empty[kStages], rfull[2], rempty[2];
+    int meta_u[kStages], meta_c[kStages];
+    int rmeta[2];
+    int seg_e[kMaxE];
+    int n_seg;
+    volatile int abort;
+    // the epilogue warp's own tables: per active expert its first row, row
+    // count and tokens; per token the x prescale
+    int ep_rbase[kMaxE];
+    uint8_t ep_cnt[kMaxE];
+    uint8_t ep_tok[kMaxE][8];
+    float ep_xs[8];
+};
+constexpr int kSmemBytes = (int)sizeof(Smem) + 1024;  // + alignment slack
+
+__device__ __forceinline__ Smem &smem_ref(uint8_t *raw) {
+    return *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ uint4 ldg128(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
+
+// bf16 rows are read by MMA row g from shared row sigma(g) (and sigma(g) + 8):
+// with the 128-byte swizzle this keeps each quarter warp's 16-byte reads on
+// distinct bank groups. The epilogue puts results back at row sigma(g).
+__device__ __forceinline__ int sigma(int g) { return (g >> 1) | ((g & 1) << 2); }
+
+struct Unit {
+    int kind, seg, tile, nst;
+};
+
+// Unit numbering: [shared gate/up][routed gate/up][shared down][routed down].
+// Shared gate/up units are assigned statically (they need no routing), routed
+// gate/up units through the work queue, and the down units as one contiguous,
+// stage-balanced range per CTA (few expert changes, so few reloads of h).
+__device__ __forceinline__ Unit unit_of(int u, int usg, int n_seg, int usd) {
+    if (u < usg) return Unit{kGsh, -1, u, 8};
+    int r = u - usg;
+    if (r < n_seg * kGuTiles) return Unit{kGrt, r / kGuTiles, r % kGuTiles, 2};
+    r -= n_seg * kGuTiles;
+    if (r < usd) return Unit{kDsh, -1, r, 2};
+    r -= usd;
+    return Unit{kDrt, r / kDnTiles, r % kDnTiles, 1};
+}
+
+__device__ __forceinline__ void fail(const DecodeArgs &a, Smem &s) {
+    set_device_error(a.err, MOE_DEVERR_TIMEOUT);
+    s.abort = 1;
+}
+
+// Bounded wait until *p >= target (another CTA's release). Lane 0 polls with
+// backoff; every lane then acquires for itself.
+__device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t target, int lane) {
+    bool ok = true;
+    if (lane == 0 && ld_acquire(p) < target) {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire(p) < target) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) { ok = false; break; }
+            __nanosleep(256);
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) ld_acquire(p);
+    return ok;
+}
+
+__device__ __forceinline__ void arm(Smem &s, int slot, int u, int c, uint32_t tx) {
+    s.meta_u[slot] = u;
+    s.meta_c[slot] = c;
+    mbar_arrive_expect_tx(&s.full[slot], tx);
+}
+
+// One 32-block of MXFP4 rows (r0 + g, r0 + g + 8 of a box with `rows` rows,
+// block = 16-byte unit `unit` of chunk `chunk`) against B.
+__device__ __forceinline__ void mxfp4_block(float acc[4], const uint8_t *box, int rows, int chunk, int unit, int r0,
+                                            int g, int q, uint32_t sw_lo, uint32_t sw_hi, int sj,
+                                            const uint32_t b[4]) {
+    uint32_t al[4], ah[4];
+    e2m1x8_to_f16x8(lds32(box + swz_off(chunk, rows, r0 + g, unit) + 4 * q), al);
+    e2m1x8_to_f16x8(lds32(box + swz_off(chunk, rows, r0 + g + 8, unit) + 4 * q), ah);
+    float t[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_f16_16816(t, al[0], ah[0], al[1], ah[1], b[0], b[1]);
+    mma_f16_16816(t, al[2], ah[2], al[3], ah[3], b[2], b[3]);
+    const float sl = e8m0_fast(sw_lo, sj), sh = e8m0_fast(sw_hi, sj);
+    acc[0] = fmaf(sl, t[0], acc[0]);
+    acc[1] = fmaf(sl, t[1], acc[1]);
+    acc[2] = fmaf(sh, t[2], acc[2]);
+    acc[3] = fmaf(sh, t[3], acc[3]);
+}
+
+// One 32-block (64 bytes: units 4*(kb%2)..+3 of chunk kb/2) of bf16 rows
+// sigma(g), sigma(g) + 8 against B (bf16).
+__device__ __forceinline__ void bf16_block(float acc[4], const uint8_t *box, int rows, int kb, int g, int q,
+                                           const uint32_t b[4]) {
+    const int r = sigma(g), c = kb >> 1, u = 4 * (kb & 1) + q;
+    const uint4 r0 = lds128(box + swz_off(c, rows, r, u));
+    const uint4 r1 = lds128(box + swz_off(c, rows, r + 8, u));
+    mma_bf16_16816(acc, r0.x, r1.x, r0.y, r1.y, b[0], b[1]);
+    mma_bf16_16816(acc, r0.z, r1.z, r0.w, r1.w, b[2], b[3]);
+}
+
+// C fragment -> partial tile [row][column]; MMA rows g, g + 8 land at rows
+// rg, rg + 8.
+__device__ __forceinline__ void put_partial(float *r, int rg, int q, const float acc[4]) {
+    r[rg * 8 + 2 * q] = acc[0];
+    r[rg * 8 + 2 * q + 1] = acc[1];
+    r[(rg + 8) * 8 + 2 * q] = acc[2];
+    r[(rg + 8) * 8 + 2 * q + 1] = acc[3];
+}
+
+// bf16 pair -> f16 pair scaled by an exact power of two.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, float sc) {
+    return f32x2_to_f16x2(__uint_as_float(v << 16) * sc, __uint_as_float(v & 0xFFFF0000u) * sc);
+}
+
+__device__ __forceinline__ float row_scale(uint32_t hm) {  // 2^p with max |h| * 2^-p in [2^14, 2^15)
+    return ldexpf(1.0f, hm ? floor_log2_f32(__uint_as_float(hm)) - 14 : 0);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_constant__ DecodeArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &s = smem_ref(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == kProducer * 32) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], kCW);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.rfull[i], kCW * 32);
+            mbar_init(&s.rempty[i], 1);
+        }
+        s.abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    grid_dep_launch();
+    const int usg = a.Fs > 0 ? a.Fs / 16 : 0;  // shared gate/up units (no routing needed)
+    const int usd = a.Fs > 0 ? kDshTiles : 0;
+    // finished gate/up units, published once per CTA (flush marker below);
+    // down units wait for all of them
+    uint32_t *gu_done = a.counters + 1;
+
+    // ------------------------------ producer ------------------------------
+    if (warp == kProducer) {
+        int gi = 0;
+        auto issue = [&](int u, const Unit &un) {
+            int row0 = 0;
+            if (un.kind == kGrt) row0 = s.seg_e[un.seg] * kF + 16 * un.tile;
+            if (un.kind == kDrt) row0 = s.seg_e[un.seg] * kD + 32 * un.tile;
+            for (int c = 0; c < un.nst && !s.abort; ++c, ++gi) {
+                const int slot = gi % kStages;
+                if (!mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1)) { fail(a, s); return; }
+                uint8_t *w = s.w[slot];
+                uint64_t *bar = &s.full[slot];
+                switch (un.kind) {
+                    case kGsh:
+                        arm(s, slot, u, c, 2 * 16384);
+                        tma_load_3d(w, &a.ms1, 0, 16 * un.tile, 8 * c, bar);
+                        tma_load_3d(w + 16384, &a.ms3, 0, 16 * un.tile, 8 * c, bar);
+                        break;
+                    case kGrt:
+                        arm(s, slot, u, c, 2 * 16384 + 2 * 1024);
+                        tma_load_3d(w, &a.m1c, 0, row0, 8 * c, bar);
+                        tma_load_3d(w + 16384, &a.m3c, 0, row0, 8 * c, bar);
+                        tma_load_2d(s.s[slot], &a.m1s, 64 * c, row0, bar);
+                        tma_load_2d(s.s[slot] + 1024, &a.m3s, 64 * c, row0, bar);
+                        break;
+                    case kDsh:
+                        arm(s, slot, u, c, 32768);
+                        tma_load_3d(w, &a.ms2, 0, 16 * un.tile, 16 * c, bar);
+                        break;
+                    default:
+                        arm(s, slot, u, c, 32768 + 2048);
+                        tma_load_3d(w, &a.m2c, 0, row0, 0, bar);
+                        tma_load_2d(s.s[slot], &a.m2s, 0, row0, bar);
+                }
+            }
+        };
+        if (lane == 0) {
+            prefetch_tensormap(&a.m1c);
+            prefetch_tensormap(&a.m2c);
+            for (int u = blockIdx.x; u < usg && !s.abort; u += gridDim.x) issue(u, unit_of(u, usg, 0, 0));
+        }
+        __syncwarp();
+        grid_dep_wait();  // routing results and zeroed counters from here on
+        int n = 0;        // active experts, ascending
+        for (int e0 = 0; e0 < a.E; e0 += 32) {
+            const int e = e0 + lane;
+            const bool act = e < a.E && a.offsets[e + 1] > a.offsets[e];
+            const unsigned m = __ballot_sync(0xffffffffu, act);
+            if (act) s.seg_e[n + __popc(m & ((1u << lane) - 1u))] = e;
+            n += __popc(m);
+        }
+        if (lane != 0) return;
+        s.n_seg = n;
+        const int gu_end = usg + n * kGuTiles;
+        // Routed gate/up: the first three quarters as one static, stage-balanced
+        // range per CTA (no atomics; CTAs that carry a shared unit take 8 fewer
+        // stages), the last quarter from the queue in chunks of kGrab, which
+        // evens out CTAs that started late or ran slow. Falls back to the
+        // queue alone when the static split would not be monotonic.
+        const int R = n * kGuTiles;
+        int Rs = R - R / 4;
+        const long long tot = 8ll * usg + 2ll * Rs;
+        if (usg > (int)gridDim.x || tot < 8ll * gridDim.x) Rs = 0;
+        auto rstart = [&](int b) {
+            const long long st = tot * b / gridDim.x - 8ll * min(b, usg);
+            return (int)min((long long)Rs, max(0ll, (st + 1) / 2));
+        };
+        const int rs0 = Rs ? rstart(blockIdx.x) : 0, rs1 = Rs ? rstart(blockIdx.x + 1) : 0;
+        for (int u = usg + rs0; u < usg + rs1 && !s.abort; ++u) issue(u, unit_of(u, usg, n, usd));
+        constexpr int kGrab = 2;
+        int next = usg + Rs + (int)atomicAdd(a.counters, (uint32_t)kGrab);
+        while (!s.abort) {  // the next chunk is fetched one chunk ahead
+            const int u0 = next;
+            if (u0 >= gu_end) break;
+            next = usg + Rs + (int)atomicAdd(a.counters, (uint32_t)kGrab);
+            for (int u = u0; u < min(u0 + kGrab, gu_end) && !s.abort; ++u) issue(u, unit_of(u, usg, n, usd));
+        }
+        // this CTA's contiguous share of the down units (shared tiles cost 2 stages)
+        const long long cost = 2ll * usd + (long long)n * kDnTiles;
+        auto first = [&](long long cst) {
+            return gu_end + (cst <= 2ll * usd ? (int)((cst + 1) / 2) : usd + (int)(cst - 2ll * usd));
+        };
+        const int d0 = first(cost * blockIdx.x / gridDim.x), d1 = first(cost * (blockIdx.x + 1) / gridDim.x);
+        for (int u = d0; u < d1 && !s.abort; ++u) issue(u, unit_of(u, usg, n, usd));
+        if (!s.abort) {
+            const int slot = gi % kStages;
+            if (mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1)) {
+                s.meta_u[slot] = -1;
+                mbar_arrive(&s.full[slot]);
+            } else {
+                fail(a, s);
+            }
+            ++gi;
+        }
+        for (int g = gi - kStages; g < gi; ++g)  // copies in flight finish before exit
+            if (g >= 0) mbar_wait(&s.full[g % kStages], (g / kStages) & 1);
+        return;
+    }
+
+    // ------------------------------ epilogue ------------------------------
+    if (warp == kEpilogue) {
+        grid_dep_wait();
+        // per-expert tables, same ascending order as the producer's list
+        int n = 0;
+        for (int e0 = 0; e0 < a.E; e0 += 32) {
+            const int e = e0 + lane;
+            const bool act = e < a.E && a.offsets[e + 1] > a.offsets[e];
+            const unsigned m = __ballot_sync(0xffffffffu, act);
+            if (act) {
+                const int sg = n + __popc(m & ((1u << lane) - 1u));
+                s.ep_rbase[sg] = a.offsets[e];
+                s.ep_cnt[sg] = (uint8_t)(a.offsets[e + 1] - a.offsets[e]);
+            }
+            n += __popc(m);
+        }
+        __syncwarp();
+        for (int sg = lane; sg < n; sg += 32)
+            for (int i = 0; i < s.ep_cnt[sg]; ++i) s.ep_tok[sg][i] = (uint8_t)(a.perm[s.ep_rbase[sg] + i] / a.k);
+        if (lane < a.T) s.ep_xs[lane] = a.xscale[lane].x;
+        __syncwarp();
+        uint32_t finished = 0;  // gate/up units finished here and not yet published
+        int dseg = -1;
+        float dsc = 1.f;        // lane i < 8: output scale of row i of segment dseg
+        for (int ru = 0;; ++ru) {
+            const int rb = ru & 1;
+            if (!mbar_wait(&s.rfull[rb], (ru >> 1) & 1)) { fail(a, s); return; }
+            const int m = s.rmeta[rb];
+            if (m == -1) return;
+            if (m == -2) {  // publish: this CTA's h / hs writes, then its count
+                __threadfence();
+                __syncwarp();
+                if (lane == 0 && finished) atomicAdd(gu_done, finished);
+                finished = 0;
+                if (lane == 0) mbar_arrive(&s.rempty[rb]);
+                continue;
+            }
+            const Unit un = unit_of(m >> 3, usg, n, usd);
+            const float(*red)[2][128] = s.red[rb];
+            if (un.kind == kGsh || un.kind == kGrt) {
+                const bool sh = un.kind == kGsh;
+                const int rbase = sh ? 0 : s.ep_rbase[un.seg], cnt = sh ? a.T : s.ep_cnt[un.seg];
+                for (int o = lane; o < 16 * 8; o += 32) {
+                    const int row = o & 15, i = o >> 4;  // i: token (shared) or row of the expert (routed)
+                    uint32_t hb = 0;
+                    if (i < cnt) {
+                        const int tok = sh ? i : s.ep_tok[un.seg][i];
+                        float gs = 0.f, us = 0.f;
+#pragma unroll
+                        for (int w = 0; w < kCW; ++w) {
+                            gs += red[w][0][row * 8 + tok];
+                            us += red[w][1][row * 8 + tok];
+                        }
+                        if (!sh) {
+                            gs *= s.ep_xs[tok];
+                            us *= s.ep_xs[tok];
+                        }
+                        hb = f32_to_bf16_rne(silu_f32(gs) * us);
+                        const int col = 16 * un.tile + row;
+                        if (sh) a.hs[(int64_t)tok * a.Fs + col] = (uint16_t)hb;
+                        else a.h[(int64_t)(rbase + i) * kF + col] = (uint16_t)hb;
+                    }
+                    if (!sh) {  // one atomic per (row of the expert) per half-warp
+                        uint32_t mx = (hb & 0x7FFFu) << 16;
+#pragma unroll
+                        for (int off = 8; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                        if ((lane & 15) == 0 && i < cnt) atomicMax(&a.hmax[rbase + i], mx);
+                    }
+                }
+                ++finished;
+            } else if (un.kind == kDsh) {
+                for (int o = lane; o < 16 * a.T; o += 32) {
+                    const int row = o & 15, tok = o >> 4;
+                    float v = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kCW; ++w) v += red[w][0][row * 8 + tok];
+                    a.shared_out[(int64_t)tok * kD + 16 * un.tile + row] = v;
+                }
+            } else {
+                const int rbase = s.ep_rbase[un.seg], cnt = s.ep_cnt[un.seg];
+                if (un.seg != dseg) {
+                    dseg = un.seg;
+                    dsc = lane < cnt ? row_scale(__ldcg(&a.hmax[rbase + lane])) : 1.f;
+                }
+                for (int o = lane; o < 32 * 8; o += 32) {
+                    const int row = o & 31, i = o >> 5;
+                    const float sc = __shfl_sync(0xffffffffu, dsc, i);
+                    if (i < cnt) {
+                        float v = 0.f;
+#pragma unroll
+                        for (int w = 0; w < kCW; ++w) v += red[w][row >> 4][(row & 15) * 8 + i];
+                        a.out_rows[(int64_t)(rbase + i) * kD + 32 * un.tile + row] = v * sc;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.rempty[rb]);
+        }
+    }
+
+    // ------------------------------ consumers ------------------------------
+    const int g = lane >> 2, q = lane & 3;
+    uint32_t B[16][4];
+    int bkind = -1, bseg = -2;  // what B holds
+    bool dep = false;           // grid dependency resolved for this thread
+    bool flushed = false;       // gate/up count of this CTA published
+    float acc[2][4];
+    int ru = 0;
+    auto marker = [&](int m) {  // a hand-off without a tile: -1 end, -2 publish
+        const int rb = ru & 1;
+        if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) return false;
+        if (threadIdx.x == 0) s.rmeta[rb] = m;
+        mbar_arrive(&s.rfull[rb]);
+        ++ru;
+        return true;
+    };
+    for (int gi = 0;; ++gi) {
+        const int slot = gi % kStages;
+        if (!mbar_wait(&s.full[slot], (gi / kStages) & 1)) { fail(a, s); return; }
+        const int u = s.meta_u[slot], c = s.meta_c[slot];
+        if (u < 0) {  // end of work: publish (if still due) and tell the epilogue
+            if ((!flushed && !marker(-2)) || !marker(-1)) fail(a, s);
+            return;
+        }
+        const Unit un = unit_of(u, usg, u < usg ? 0 : s.n_seg, usd);
+        if (un.kind != kGsh && !dep) {
+            grid_dep_wait();
+            dep = true;
+        }
+        if (un.kind != bkind || un.seg != bseg) {
+            bkind = un.kind;
+            bseg = un.seg;
+            if (un.kind == kDsh || un.kind == kDrt) {  // every gate/up unit must be complete
+                if (!flushed) {
+                    if (!marker(-2)) { fail(a, s); return; }
+                    flushed = true;
+                }
+                if (!wait_count(gu_done, (uint32_t)(usg + s.n_seg * kGuTiles), lane)) { fail(a, s); return; }
+            }
+            if (un.kind == kGsh || un.kind == kGrt) {
+                const bool sh = un.kind == kGsh;
+                const int tok = min(g, a.T - 1);
+                const float inv = sh ? 1.f : a.xscale[tok].y;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    // shared: stage j/2 holds blocks 16(j/2)..+15 of K; this warp takes 2w, 2w+1
+                    // routed: stage j/8 holds blocks 64(j/8)..+63; this warp takes 8w..8w+7
+                    const int kb = sh ? 16 * (j / 2) + 2 * warp + (j & 1) : 64 * (j / 8) + 8 * warp + (j & 7);
+                    const uint4 v = ldg128(a.x + (int64_t)tok * kD + 32 * kb + 8 * q);
+                    const uint32_t raw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) B[j][i] = sh ? raw[i] : bf16x2_to_f16x2(raw[i], inv);
+                }
+            } else if (un.kind == kDsh) {
+                const int tok = min(g, a.T - 1);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {  // stage j/4 holds blocks 32(j/4)..+31; this warp 4w..4w+3
+                    const uint4 v = ldcg128(a.hs + (int64_t)tok * a.Fs + 32 * (32 * (j / 4) + 4 * warp + (j & 3)) + 8 * q);
+                    B[j][0] = v.x; B[j][1] = v.y; B[j][2] = v.z; B[j][3] = v.w;
+                }
+            } else {
+                const int e = s.seg_e[un.seg];
+                const int rbase = a.offsets[e], cnt = a.offsets[e + 1] - rbase;
+                const int row = rbase + min(g, cnt - 1);
+                const float sc = 1.0f / row_scale(__ldcg(&a.hmax[row]));
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 v = ldcg128(a.h + (int64_t)row * kF + 32 * (8 * warp + j) + 8 * q);
+                    B[j][0] = bf16x2_to_f16x2(v.x, sc);
+                    B[j][1] = bf16x2_to_f16x2(v.y, sc);
+                    B[j][2] = bf16x2_to_f16x2(v.z, sc);
+                    B[j][3] = bf16x2_to_f16x2(v.w, sc);
+                }
+            }
+        }
+        if (c == 0 || un.kind == kDrt)
+#pragma unroll
+            for (int m = 0; m < 2; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+        const uint8_t *st = s.w[slot], *ss = s.s[slot];
+        if (un.kind == kGsh) {
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+                if (cc == c)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+                        for (int m = 0; m < 2; ++m)
+                            bf16_block(acc[m], st + 16384 * m, 16, 2 * warp + jj, g, q, B[2 * cc + jj]);
+        } else if (un.kind == kGrt) {
+            uint32_t sw[2][2][2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) sw[m][hh][i] = lds32(ss + 1024 * m + (g + 8 * hh) * 64 + 4 * (2 * warp + i));
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc)
+                if (cc == c)
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                        for (int m = 0; m < 2; ++m)
+                            mxfp4_block(acc[m], st + 16384 * m, 16, warp, jj, 0, g, q, sw[m][0][jj / 4],
+                                        sw[m][1][jj / 4], jj % 4, B[8 * cc + jj]);
+        } else if (un.kind == kDsh) {
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc)
+                if (cc == c)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) bf16_block(acc[0], st, 16, 4 * warp + jj, g, q, B[4 * cc + jj]);
+        } else {
+            uint32_t sw[2][2][2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) sw[t][hh][i] = lds32(ss + (16 * t + g + 8 * hh) * 64 + 4 * (2 * warp + i));
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+                    mxfp4_block(acc[t], st, 32, warp, jj, 16 * t, g, q, sw[t][0][jj / 4], sw[t][1][jj / 4], jj % 4,
+                                B[jj]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[slot]);
+        const bool last = un.kind == kDrt || c == un.nst - 1;
+        if (last) {  // hand the unit (or tile) to the epilogue warp
+            const int rb = ru & 1;
+            if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
+            const int rg = (un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;  // bf16 tiles read rows sigma(g)
+            put_partial(s.red[rb][warp][0], rg, q, acc[0]);
+            if (un.kind != kDsh) put_partial(s.red[rb][warp][1], rg, q, acc[1]);
+            if (threadIdx.x == 0) s.rmeta[rb] = u * 8 + c;
+            mbar_arrive(&s.rfull[rb]);
+            ++ru;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Decode routing: fixed-order fp32 logits (one warp per expert, lane = chunk,
+// all T tokens at once; CTA 0 also computes the per-token f16 prescale), then
+// one CTA does top-k, softmax gates, histogram / scan / permutation and
+// resets the FFN kernel's scratch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int xs_index(int t, int c, int v) { return (t * 32 + c) * 17 + v; }  // padded [T][32][17] uint4
+
+__global__ void __launch_bounds__(128) decode_logits_kernel(const uint16_t *__restrict__ x,
+                                                            const uint16_t *__restrict__ wr,
+                                                            const float *__restrict__ bias, int T, int E,
+                                                            float *__restrict__ logits, float2 *__restrict__ xscale) {
+    extern __shared__ uint4 xs4[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 4 + warp;
+    constexpr int chunk = kD / 32;  // 128 elements = 16 uint4 per lane
+    uint4 wv[16];
+    if (e < E)
+#pragma unroll
+        for (int v = 0; v < 16; ++v) wv[v] = ldg128(wr + (int64_t)e * kD + lane * chunk + 8 * v);
+    for (int i = threadIdx.x; i < T * 512; i += blockDim.x) xs4[xs_index(i / 512, (i / 16) % 32, i % 16)] = ldg128(x + 8 * i);
+    __syncthreads();
+    grid_dep_launch();
+    if (blockIdx.x == 0)
+        for (int t = warp; t < T; t += 4) {  // per-token 2^p with max|x| 2^-p in [2^14, 2^15)
+            float mx = 0.f;
+            for (int i = lane; i < 512; i += 32) {
+                const uint4 v = xs4[xs_index(t, i / 16, i % 16)];
+                const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(r[j] << 16)), fabsf(__uint_as_float(r[j] & 0xFFFF0000u))));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) {
+                const int p = mx > 0.f ? floor_log2_f32(mx) - 14 : 0;
+                xscale[t] = make_float2(ldexpf(1.0f, p), ldexpf(1.0f, -p));
+            }
+        }
+    if (e >= E) return;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+        const uint32_t wa[4] = {wv[v].x, wv[v].y, wv[v].z, wv[v].w};
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+            if (t < T) {
+                const uint4 xv = xs4[xs_index(t, lane, v)];
+                const uint32_t xa[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    acc[t] = __fmaf_rn(__uint_as_float(xa[qq] << 16), __uint_as_float(wa[qq] << 16), acc[t]);
+                    acc[t] = __fmaf_rn(__uint_as_float(xa[qq] & 0xFFFF0000u), __uint_as_float(wa[qq] & 0xFFFF0000u), acc[t]);
+                }
+            }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+        if (t < T) {
+            float v = acc[t];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0) logits[(int64_t)t * E + e] = bias ? __fadd_rn(v, bias[e]) : v;
+        }
+}
+
+__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
+    const bool na = isnan(va), nb = isnan(vb);
+    if (na != nb) return nb;
+    if (!na && va != vb) return va > vb;
+    return ia < ib;
+}
+
+struct FinalizeArgs {
+    int T, E, k;
+    const float *logits;
+    int32_t *idx, *counts, *offsets, *perm, *inv_perm;
+    float *gates;
+    uint32_t *hmax, *counters;
+};
+
+__global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs a) {
+    __shared__ float lg[8 * kMaxE];
+    __shared__ int hist[kMaxE];
+    __shared__ int sidx[256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = a.T, E = a.E, k = a.k;
+    grid_dep_launch();
+    for (int i = threadIdx.x; i < E + 2; i += blockDim.x) a.counters[i] = 0u;
+    for (int i = threadIdx.x; i < T * k; i += blockDim.x) a.hmax[i] = 0u;
+    grid_dep_wait();
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) lg[i] = a.logits[i];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    if (warp < T) {  // top-k + gates of token `warp`
+        const float *l = lg + warp * E;
+        uint32_t taken = 0;
+        float my_l = 0.f, l0v = 0.f;
+        int my_e = -1;
+        for (int j = 0; j < k; ++j) {
+            float bv = 0.f;
+            int bi = -1;
+            for (int i = 0, e = lane; e < E; ++i, e += 32) {
+                if (taken >> i & 1u) continue;
+                const float v = l[e];
+                if (bi < 0 || ranks_before(v, e, bv, bi)) { bv = v; bi = e; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (oi >= 0 && (bi < 0 || ranks_before(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+            }
+            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (j == 0) l0v = bv;
+            if (lane == j) { my_l = bv; my_e = bi; }
+        }
+        const float ex = lane < k ? expf(my_l - l0v) : 0.f;
+        const float den = warp_sum(ex);
+        if (lane < k) {
+            a.idx[warp * k + lane] = my_e;
+            a.gates[warp * k + lane] = ex / den;
+            sidx[warp * k + lane] = my_e;
+        }
+    }
+    __syncthreads();
+    const int S = T * k;
+    if (threadIdx.x < S) atomicAdd(&hist[sidx[threadIdx.x]], 1);
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan over experts
+        int run = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int c = e < E ? hist[e] : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (e < E) {
+                a.counts[e] = c;
+                a.offsets[e] = run + incl - c;
+                hist[e] = run + incl - c;  // first row of expert e
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) a.offsets[E] = run;
+    }
+    __syncthreads();
+    if (threadIdx.x < S) {  // stable rank: earlier slots of the same expert
+        const int s0 = threadIdx.x, e = sidx[s0];
+        int r = 0;
+        for (int s1 = 0; s1 < s0; ++s1) r += (sidx[s1] == e);
+        const int row = hist[e] + r;
+        a.perm[row] = s0;
+        a.inv_perm[s0] = row;
+    }
+}
+
+// Stage-API entry (no routing in this call): the x prescale and the scratch reset.
+__global__ void __launch_bounds__(256) decode_prep_kernel(const uint16_t *__restrict__ x, int T, int S, int E,
+                                                          float2 *xscale, uint32_t *hmax, uint32_t *counters) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < T) {
+        float mx = 0.f;
+        for (int i = lane; i < kD / 8; i += 32) {
+            const uint4 v = ldg128(x + (int64_t)warp * kD + 8 * i);
+            const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(r[j] << 16)), fabsf(__uint_as_float(r[j] & 0xFFFF0000u))));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) {
+            const int p = mx > 0.f ? floor_log2_f32(mx) - 14 : 0;
+            xscale[warp] = make_float2(ldexpf(1.0f, p), ldexpf(1.0f, -p));
+        }
+    }
+    for (int i = threadIdx.x; i < S; i += blockDim.x) hmax[i] = 0u;
+    for (int i = threadIdx.x; i < E + 2; i += blockDim.x) counters[i] = 0u;
+}
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+constexpr int kLogitsSmem = 8 * 32 * 17 * 16;
+
+cudaError_t set_smem_attrs() {
+    static bool done[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (done[dev]) return cudaSuccess;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(decode_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)))
+        return e;
+    if ((e = cudaFuncSetAttribute(decode_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLogitsSmem)))
+        return e;
+    done[dev] = true;
+    return cudaSuccess;
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// its predecessor in the stream finishes; it calls griddepcontrol.wait before
+// reading that predecessor's results.
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
+}  // namespace
+
+bool decode_path_applies(const moe_dims &d) {
+    // the tiling is written for d_model 4096, d_ff 2048 (and a shared d_ff of 2048)
+    return d.T >= 1 && d.T <= 8 && d.wfmt == MOE_W_MXFP4 && d.act == MOE_A_BF16 && d.d_model == kD &&
+           d.d_ff == kF && (d.d_ff_shared == 0 || d.d_ff_shared == 2048) && d.E <= kMaxE;
+}
+
+bool decode_route_applies(const moe_dims &d) {
+    return decode_path_applies(d) && d.route == MOE_ROUTE_SOFTMAX_TOPK && d.T * d.k <= 256;
+}
+
+// Decode routing: logits kernel + finalize kernel (top-k, permute, scratch
+// reset for the FFN kernel). The logits kernel also writes the x prescale.
+cudaError_t launch_decode_route(const moe_dims &d, const uint16_t *x, const moe_weights &w, int32_t *idx,
+                                float *gates, int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm,
+                                uint8_t *ws, const WsLayout &L, cudaStream_t s) {
+    cudaError_t e = set_smem_attrs();
+    if (e != cudaSuccess) return e;
+    float *logits = reinterpret_cast<float *>(ws + L.logits);
+    decode_logits_kernel<<<ceil_div(d.E, 4), 128, kLogitsSmem, s>>>(x, w.w_router, w.router_bias, d.T, d.E, logits,
+                                                                    reinterpret_cast<float2 *>(ws + L.xscale));
+    FinalizeArgs f;
+    f.T = d.T; f.E = d.E; f.k = d.k; f.logits = logits;
+    f.idx = idx; f.counts = counts; f.offsets = offsets; f.perm = perm; f.inv_perm = inv_perm; f.gates = gates;
+    f.hmax = reinterpret_cast<uint32_t *>(ws + L.hmax);
+    f.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
+    if ((e = launch_pdl(decode_finalize_kernel, dim3(1), dim3(256), 0, s, f)) != cudaSuccess) return e;
+    count_launches(2);
+    return cudaGetLastError();
+}
+
+// Routed + shared expert FFN for decode batches in one launch. `shared_out`
+// may be null. `prepared`: the decode routing already ran on this workspace
+// (x prescale, scratch reset); otherwise a small kernel does that first.
+cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
+                              const int32_t *perm, float *out_rows, float *shared_out, uint8_t *ws,
+                              const WsLayout &L, cudaStream_t s, bool prepared) {
+    cudaError_t e = set_smem_attrs();
+    if (e != cudaSuccess) return e;
+    const Mxfp4Layout L1 = mxfp4_layout(d, MOE_MAT_W1), L2 = mxfp4_layout(d, MOE_MAT_W2);
+    DecodeArgs a;
+    memset(&a, 0, sizeof a);
+    const uint8_t *p1 = static_cast<const uint8_t *>(w.w1), *p3 = static_cast<const uint8_t *>(w.w3),
+                  *p2 = static_cast<const uint8_t *>(w.w2);
+    const uint64_t r13 = (uint64_t)d.E * kF, r2 = (uint64_t)d.E * kD;
+    bool ok = make_chunked_map(&a.m1c, p1 + L1.codes, r13, kD / 2, 16, 8) &&
+              make_chunked_map(&a.m3c, p3 + L1.codes, r13, kD / 2, 16, 8) &&
+              make_chunked_map(&a.m2c, p2 + L2.codes, r2, kF / 2, 32, 8) &&
+              make_plain_map(&a.m1s, p1 + L1.srow, r13, kD / 32, 64, 16) &&
+              make_plain_map(&a.m3s, p3 + L1.srow, r13, kD / 32, 64, 16) &&
+              make_plain_map(&a.m2s, p2 + L2.srow, r2, kF / 32, 64, 32);
+    if (ok && shared_out)
+        ok = make_chunked_map(&a.ms1, w.sw1, d.d_ff_shared, kD * 2, 16, 8) &&
+             make_chunked_map(&a.ms3, w.sw3, d.d_ff_shared, kD * 2, 16, 8) &&
+             make_chunked_map(&a.ms2, w.sw2, kD, d.d_ff_shared * 2, 16, 16);
+    if (!ok) return cudaErrorInvalidValue;
+    a.T = d.T; a.E = d.E; a.k = d.k;
+    a.Fs = shared_out ? d.d_ff_shared : 0;
+    a.offsets = offsets; a.perm = perm; a.x = x;
+    a.xscale = reinterpret_cast<const float2 *>(ws + L.xscale);
+    a.h = reinterpret_cast<uint16_t *>(ws + L.h);
+    a.hmax = reinterpret_cast<uint32_t *>(ws + L.hmax);
+    a.hs = reinterpret_cast<uint16_t *>(ws + L.sh_h);
+    a.out_rows = out_rows;
+    a.shared_out = shared_out;
+    a.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
+    a.err = device_error_word();
+    if (!prepared) {
+        decode_prep_kernel<<<1, 256, 0, s>>>(x, d.T, d.T * d.k, d.E, reinterpret_cast<float2 *>(ws + L.xscale), a.hmax,
+                                              a.counters);
+        count_launches(1);
+    }
+    if ((e = launch_pdl(decode_ffn_kernel, dim3(num_sms()), dim3(kThreads), kSmemBytes, s, a)) != cudaSuccess)
+        return e;
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

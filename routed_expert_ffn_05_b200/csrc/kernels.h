@@ -26,8 +26,9 @@ cudaError_t launch_permute(const moe_dims &d, const int32_t *idx, int32_t *count
                            int32_t *perm, int32_t *inv_perm, int32_t *blkcnt, int32_t *blkbase,
                            int64_t nblk, cudaStream_t s);
 
+// `pdl`: launch programmatically after the preceding kernel (the decode FFN).
 cudaError_t launch_combine(const moe_dims &d, const float *out_rows, const int32_t *inv_perm,
-                           const float *gates, const float *shared, float *y, cudaStream_t s);
+                           const float *gates, const float *shared, float *y, cudaStream_t s, bool pdl = false);
 
 cudaError_t launch_quantize_weights(const moe_dims &d, int which, const float *w, uint8_t *canonical,
                                     cudaStream_t s);
@@ -40,10 +41,23 @@ cudaError_t launch_quant_act_bf16(const uint16_t *x, int64_t rows, int K, uint8_
 cudaError_t launch_quant_act_f32(const float *x, int64_t rows, int K, uint8_t *codes, uint8_t *scales,
                                  cudaStream_t s);
 
-// Routed expert FFN over all permuted rows; ws gives h / h8 / x8 scratch.
+// Routed expert FFN over all permuted rows (ws gives h / h8 / x8 scratch), and
+// the shared expert into `shared_out` when it is non-null.
+// `prepared`: the fused decode routing kernel already ran on this workspace.
 cudaError_t launch_expert_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x,
                               const int32_t *offsets, const int32_t *perm, float *out_rows,
-                              uint8_t *ws, const WsLayout &L, cudaStream_t s);
+                              float *shared_out, uint8_t *ws, const WsLayout &L, cudaStream_t s,
+                              bool prepared = false);
+
+// Decode-sized path (tensor-core GEMV over streamed weights), when it applies.
+bool decode_path_applies(const moe_dims &d);
+bool decode_route_applies(const moe_dims &d);
+cudaError_t launch_decode_route(const moe_dims &d, const uint16_t *x, const moe_weights &w, int32_t *idx,
+                                float *gates, int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm,
+                                uint8_t *ws, const WsLayout &L, cudaStream_t s);
+cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
+                              const int32_t *perm, float *out_rows, float *shared_out, uint8_t *ws,
+                              const WsLayout &L, cudaStream_t s, bool prepared);
 
 cudaError_t launch_shared_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, float *out,
                               float *hbuf, cudaStream_t s);

@@ -65,7 +65,7 @@ static inline Q2kLayout q2k_layout(const moe_dims &d, int which) {
 // Workspace regions (byte offsets), one layout for every entry point.
 struct WsLayout {
     int64_t logits, topk_idx, topk_w, counts, offsets, perm, inv_perm, blkcnt, blkbase;
-    int64_t x8, xs, h, h8, hs, out_rows, sh_h, sh_out, total;
+    int64_t x8, xs, xscale, counters, h, hmax, h8, hs, out_rows, sh_h, sh_out, total;
     int64_t nblk;
 };
 static const int kPermuteBlock = 256;  // slots per permute block
@@ -87,7 +87,10 @@ static inline WsLayout ws_layout(const moe_dims &d) {
     w.blkbase = take(w.nblk * E * 4);
     w.x8 = take(T * dm);
     w.xs = take(T * dm / 32);
+    w.xscale = take(T * 8);
+    w.counters = take((E + 2) * 4);  // work queue, shared gate/up done, per-expert done
     w.h = take(S * F * 4);
+    w.hmax = take(S * 4);
     w.h8 = take(S * F);
     w.hs = take(S * F / 32);
     w.out_rows = take(S * dm * 4);

@@ -1,0 +1,25 @@
+// Host-side TMA tensor maps (cuTensorMapEncodeTiled through the runtime's
+// driver entry point, so the library needs no link against libcuda).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// A row-major byte matrix [rows][row_bytes] seen as 3D (128-byte chunk,
+// row, chunk index) with 128-byte swizzle. A box of (128, box_rows,
+// box_chunks) lands in shared memory as [chunk][row][128 B] with 16-byte unit
+// u of row r stored at unit u ^ (r % 8): threads reading the same unit of 8
+// consecutive rows hit 8 different bank groups. Base 16-byte aligned,
+// row_bytes a multiple of 128.
+bool make_chunked_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows,
+                      uint32_t box_chunks);
+
+// A row-major byte matrix [rows][row_bytes] as 2D without swizzle, box
+// (box_bytes, box_rows). box_bytes a multiple of 16.
+bool make_plain_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_bytes,
+                    uint32_t box_rows);
+
+}  // namespace moe
