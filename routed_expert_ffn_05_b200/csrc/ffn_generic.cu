@@ -193,6 +193,7 @@ cudaError_t launch_expert_ffn(const moe_dims &d, const moe_weights &w, const uin
     if (shared_out &&
         (e = launch_shared_ffn_generic(d, w, x, shared_out, reinterpret_cast<float *>(ws + L.sh_h), s)) != cudaSuccess)
         return e;
+    if (tc_path_applies(d)) return launch_tc_ffn(d, w, x, offsets, perm, out_rows, ws, L, s);
     return launch_expert_ffn_generic(d, w, x, offsets, perm, out_rows, ws, L, s);
 }
 

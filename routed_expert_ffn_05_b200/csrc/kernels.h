@@ -59,6 +59,11 @@ cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uin
                               const int32_t *perm, float *out_rows, float *shared_out, uint8_t *ws,
                               const WsLayout &L, cudaStream_t s, bool prepared);
 
+// w4a8 with MXFP4 weights on the tensor cores (tcgen05 block-scaled MMA).
+bool tc_path_applies(const moe_dims &d);
+cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
+                          const int32_t *perm, float *out_rows, uint8_t *ws, const WsLayout &L, cudaStream_t s);
+
 cudaError_t launch_shared_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, float *out,
                               float *hbuf, cudaStream_t s);
 

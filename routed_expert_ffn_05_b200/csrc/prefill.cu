@@ -1,0 +1,447 @@
+// Prefill-sized expert FFN in w4a8 mode on the 5th-generation tensor cores:
+// block-scaled MMA of E2M1 weights against E4M3 activations, both with E8M0
+// scales per 32 along K (OCP MX v1.0), fp32 accumulate in tensor memory.
+//
+// The routed experts are FP4 and the expert work is batched per expert ("DS4",
+// dibi8.com, "Key architectural innovations" item 1; "DwarfStar",
+// hysenlabs.com, "Model support and quantisation"). The layer's math:
+// g = W1 a, u = W3 a, h = silu(g) * u quantised to MXFP8 along F, o = W2 h.
+//
+// Mapping onto tcgen05.mma (M = 128, K = 32 per instruction):
+//  - the MMA's M side is 128 weight rows and its N side is a tile of up to
+//    128 of the expert's tokens, trimmed to a multiple of 16. Routing is
+//    skewed (a Zipf-like expert popularity leaves many experts with a few
+//    tokens), so putting tokens on N costs at most 15 padded columns per tile
+//    where 128-row token tiles on M would cost up to 127 rows;
+//  - gate/up: two MMAs per K step (W1 and W3 tiles against the same token
+//    tile) into two 128-column fp32 accumulators, so SwiGLU pairs g and u in
+//    the same thread after tcgen05.ld; the h block amax along F (across the
+//    warp's 32 lanes = 32 consecutive weight rows) is one redux.sync;
+//  - down: one MMA per K step, 128 rows of W2;
+//  - operands arrive by TMA in 128-byte-swizzled K-major boxes of 128 K; E2M1
+//    codes are expanded to one byte per element in shared memory by the
+//    tensor map's 16U4_ALIGN16B type; the E8M0 scales come in 512-byte atoms
+//    (128 rows x 4 blocks) that tcgen05.cp broadcasts into tensor memory;
+//  - one persistent CTA per SM: a TMA warp, an MMA warp and eight epilogue
+//    warps, a 4-stage mbarrier ring; every wait is bounded.
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+#include "tma.h"
+
+namespace moe {
+namespace {
+
+constexpr int kTcStages = 4;
+constexpr int kTcThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kTileBytes = 16384; // 128 rows x 128 bytes
+constexpr uint32_t kTmemCols = 512;
+constexpr int kSfCol = 256;       // scale-factor columns: 16 per stage from here
+constexpr int kTcMaxE = 1024;
+constexpr int kTile = 128;        // weight rows and tokens per tile, K per stage
+
+enum { kModeGU = 0, kModeDN = 1 };
+
+struct TcArgs {
+    CUtensorMap wa, wb;  // weights: W1 and W3 (gate/up) or W2 (down), E2M1 expanded
+    CUtensorMap act;     // activations: gathered x codes (gate/up) or h codes (down)
+    const uint8_t *sfa, *sfb;  // weight scale atoms (W1/W2, W3)
+    const uint8_t *sfact;      // activation scale atoms per token tile
+    const int32_t *offsets;    // [E+1] expert row ranges
+    const int32_t *ustart;     // [E+1] token-tile prefix
+    int E, Nw, K;              // weight rows per expert, K
+    uint8_t *h8;               // gate/up: h codes [S][F]
+    uint8_t *hsf;              // gate/up: h scale atoms [tiles][F/128][512]
+    float *out;                // down: rows [S][d]
+    int *err;
+};
+
+struct TcSmem {
+    uint8_t a[kTcStages][2][kTileBytes];
+    uint8_t b[kTcStages][kTileBytes];
+    uint8_t sf[kTcStages][3][512];
+    uint64_t full[kTcStages], empty[kTcStages], acc_full, acc_empty, mma_done;
+    uint32_t tmem_base;
+    volatile int abort;
+    int ustart[kTcMaxE + 1];
+};
+constexpr int kTcSmemBytes = (int)sizeof(TcSmem) + 1024;
+
+__device__ __forceinline__ TcSmem &tc_smem(uint8_t *raw) {
+    return *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
+struct Work {
+    int e, f, j, row0, nvalid;
+};
+
+// Work item w -> (expert, weight tile, token tile). Items of one expert are
+// ordered weight-tile-major, so CTAs running neighbouring items share the same
+// weight tile through L2.
+__device__ __forceinline__ Work work_of(int w, int ft, const int *ustart, int E, const int32_t *offsets) {
+    const int v = w / ft;
+    int lo = 0, hi = E - 1;  // largest e with ustart[e] <= v
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (ustart[mid] <= v) lo = mid;
+        else hi = mid - 1;
+    }
+    const int e = lo, nt = ustart[e + 1] - ustart[e];
+    const int local = w - ft * ustart[e];
+    Work wk;
+    wk.e = e;
+    wk.f = local / nt;
+    wk.j = local % nt;
+    wk.row0 = offsets[e] + kTile * wk.j;
+    wk.nvalid = min(kTile, offsets[e + 1] - wk.row0);
+    return wk;
+}
+
+__device__ __forceinline__ void tc_fail(const TcArgs &a, TcSmem &s) {
+    set_device_error(a.err, MOE_DEVERR_TIMEOUT);
+    s.abort = 1;
+}
+
+// Byte of the scale of (row t of a 128-row tile, 32-block q of a 128-wide K
+// atom) inside the atom: the order tcgen05.cp 32x128b.warpx4 spreads over TMEM.
+__device__ __forceinline__ int sf_atom_byte(int t, int q) { return (t & 31) * 16 + (t >> 5) * 4 + q; }
+
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+    uint32_t r;
+    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+    return r;
+}
+
+// 2^-se as an fp32 (exact for se in [-127, 126]).
+__device__ __forceinline__ float pow2_neg(int se) { return __uint_as_float((uint32_t)(127 - se) << 23); }
+
+template <int MODE>
+__global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_constant__ TcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    TcSmem &s = tc_smem(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr bool GU = MODE == kModeGU;
+    const int ft = a.Nw / kTile, kt_n = a.K / kTile;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kTcStages; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
+        }
+        mbar_init(&s.acc_full, 1);
+        mbar_init(&s.acc_empty, 8);
+        mbar_init(&s.mma_done, 1);
+        s.abort = 0;
+        fence_mbar_init();
+    }
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s.ustart[i] = a.ustart[i];
+    if (warp == 1) {
+        tmem_alloc(&s.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s.tmem_base;
+    const int n_work = ft * s.ustart[a.E];
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            prefetch_tensormap(&a.wa);
+            prefetch_tensormap(&a.act);
+            // an expanded E2M1 box credits the packed bytes it reads (8 KB), not
+            // the 16 KB it fills in shared memory
+            const uint32_t tx = (GU ? 2 : 1) * (kTileBytes / 2) + kTileBytes + (GU ? 3 : 2) * 512;
+            int it = 0;
+            for (int w = blockIdx.x; w < n_work && !s.abort; w += gridDim.x) {
+                const Work wk = work_of(w, ft, s.ustart, a.E, a.offsets);
+                const int wrow = wk.e * a.Nw + wk.f * kTile;
+                const int64_t wat = ((int64_t)wk.e * ft + wk.f) * kt_n;                    // weight atom base
+                const int64_t aat = ((int64_t)s.ustart[wk.e] + wk.j) * kt_n;              // activation atom base
+                for (int kt = 0; kt < kt_n; ++kt, ++it) {
+                    const int slot = it % kTcStages;
+                    if (!mbar_wait(&s.empty[slot], ((it / kTcStages) & 1) ^ 1)) { tc_fail(a, s); break; }
+                    uint64_t *bar = &s.full[slot];
+                    mbar_arrive_expect_tx(bar, tx);
+                    tma_load_2d(s.a[slot][0], &a.wa, kt * kTile, wrow, bar);
+                    if (GU) tma_load_2d(s.a[slot][1], &a.wb, kt * kTile, wrow, bar);
+                    tma_load_2d(s.b[slot], &a.act, kt * kTile, wk.row0, bar);
+                    bulk_g2s(s.sf[slot][0], a.sfa + (wat + kt) * 512, 512, bar);
+                    if (GU) bulk_g2s(s.sf[slot][1], a.sfb + (wat + kt) * 512, 512, bar);
+                    bulk_g2s(s.sf[slot][2], a.sfact + (aat + kt) * 512, 512, bar);
+                }
+            }
+            // copies in flight land before the CTA exits
+            for (int g = it - kTcStages; g < it; ++g)
+                if (g >= 0) mbar_wait(&s.full[g % kTcStages], (g / kTcStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            int it = 0, lw = 0;
+            for (int w = blockIdx.x; w < n_work && !s.abort; w += gridDim.x, ++lw) {
+                const Work wk = work_of(w, ft, s.ustart, a.E, a.offsets);
+                const int n16 = (wk.nvalid + 15) & ~15;
+                const uint32_t idesc = idesc_mx(5, 0, 128, n16);
+                if (!mbar_wait(&s.acc_empty, (lw & 1) ^ 1)) { tc_fail(a, s); break; }
+                tc_fence_after();
+                bool ok = true;
+                for (int kt = 0; kt < kt_n; ++kt, ++it) {
+                    const int slot = it % kTcStages;
+                    if (!mbar_wait(&s.full[slot], (it / kTcStages) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sfc = tmem + kSfCol + 16 * slot;
+                    tc_cp_sf(sfc, sdesc_sf(s.sf[slot][0]));
+                    if (GU) tc_cp_sf(sfc + 4, sdesc_sf(s.sf[slot][1]));
+                    tc_cp_sf(sfc + 8, sdesc_sf(s.sf[slot][2]));
+                    const uint64_t d0 = sdesc_sw128(s.a[slot][0]), d1 = sdesc_sw128(s.a[slot][1]),
+                                   db = sdesc_sw128(s.b[slot]);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint32_t id = idesc_sf_ids(idesc, ks, ks), acc = (kt | ks) != 0;
+                        const uint32_t sel = (uint32_t)ks << 30;
+                        tc_mma_mx(tmem, d0 + 2 * ks, db + 2 * ks, id, sfc | sel, (sfc + 8) | sel, acc);
+                        if (GU) tc_mma_mx(tmem + 128, d1 + 2 * ks, db + 2 * ks, id, (sfc + 4) | sel, (sfc + 8) | sel, acc);
+                    }
+                    tc_commit(&s.empty[slot]);  // frees the stage once these MMAs finish
+                }
+                if (!ok) { tc_fail(a, s); break; }
+                tc_commit(&s.acc_full);
+            }
+            tc_commit(&s.mma_done);
+            mbar_wait(&s.mma_done, 0);
+        }
+    } else {
+        // ------------------------------ epilogue ------------------------------
+        const int q = warp & 3;              // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;    // token columns [64 half, 64 half + 64)
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        int lw = 0;
+        // control flow stays warp-uniform: tcgen05.ld is a warp-collective
+        for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++lw) {
+            if (__shfl_sync(0xffffffffu, s.abort, 0)) break;
+            const Work wk = work_of(w, ft, s.ustart, a.E, a.offsets);
+            const bool ok = mbar_wait(&s.acc_full, lw & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) tc_fail(a, s);
+                break;
+            }
+            tc_fence_after();
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                if (c0 >= wk.nvalid) break;
+                uint32_t g[32];
+                tmem_ld32(lane_base + c0, g);
+                if (GU) {
+                    uint32_t u[32];
+                    tmem_ld32(lane_base + 128 + c0, u);
+                    tmem_wait_ld();
+                    const int fcol = wk.f * kTile + 32 * q + lane;  // this lane's h column
+                    const int64_t atom = (((int64_t)s.ustart[wk.e] + wk.j) * (a.Nw / kTile) + wk.f) * 512;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        float hv[2];
+                        int se[2];
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            const float gv = __uint_as_float(g[i + p]);
+                            hv[p] = silu_f32(gv) * __uint_as_float(u[i + p]);
+                            const uint32_t amax = warp_max_u32(__float_as_uint(hv[p]) & 0x7FFFFFFFu);
+                            if (amax == 0u) {
+                                se[p] = 0;
+                                hv[p] = 0.0f;
+                            } else {
+                                int e8 = floor_log2_f32(__uint_as_float(amax)) - 8;
+                                se[p] = e8 < -127 ? -127 : (e8 > 127 ? 127 : e8);
+                                hv[p] *= pow2_neg(se[p]);
+                            }
+                        }
+                        const uint32_t codes = f32x2_to_e4m3x2(hv[0], hv[1]);
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            const int t = c0 + i + p;
+                            if (t < wk.nvalid) {
+                                a.h8[(int64_t)(wk.row0 + t) * a.Nw + fcol] = (uint8_t)(codes >> (8 * p));
+                                if (lane == 0) a.hsf[atom + sf_atom_byte(t, q)] = (uint8_t)(se[p] + 127);
+                            }
+                        }
+                    }
+                } else {
+                    tmem_wait_ld();
+                    float *orow = a.out + (int64_t)wk.row0 * a.Nw + wk.f * kTile + 32 * q + lane;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c0 + i < wk.nvalid) orow[(int64_t)(c0 + i) * a.Nw] = __uint_as_float(g[i]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.acc_empty);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Token tiles per expert (ceil(count / 128)) and their exclusive prefix.
+__global__ void __launch_bounds__(1024) tc_plan_kernel(const int32_t *__restrict__ offsets, int E,
+                                                       int32_t *__restrict__ ustart) {
+    __shared__ int wsum[32];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    const int nt = e < E ? (offsets[e + 1] - offsets[e] + kTile - 1) / kTile : 0;
+    int incl = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int v = wsum[lane], w = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += t;
+        }
+        wsum[lane] = w - v;  // exclusive warp prefix
+    }
+    __syncthreads();
+    const int excl = wsum[warp] + incl - nt;
+    if (e < E) ustart[e] = excl;
+    if (e == E - 1) ustart[E] = excl + nt;
+}
+
+// One warp per permuted row: x of the row's token -> MXFP8 (E4M3 codes and
+// E8M0 scales per 32 along d, the OCP rule: scale exponent floor(log2 amax) - 8,
+// RNE, saturating; an all-zero block gets scale 127 and zero codes). Codes go
+// to the row in expert order, scales to the row's token-tile atom.
+__global__ void __launch_bounds__(256) tc_gather_quant_kernel(const uint16_t *__restrict__ x,
+                                                              const int32_t *__restrict__ offsets,
+                                                              const int32_t *__restrict__ perm,
+                                                              const int32_t *__restrict__ ustart, int S, int E,
+                                                              int k, int d, uint8_t *__restrict__ x8,
+                                                              uint8_t *__restrict__ xsf) {
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (row >= S) return;
+    const int e = expert_of_row(offsets, E, row);
+    const int r = row - offsets[e];
+    const int tok = perm[row] / k;
+    const int64_t atom0 = ((int64_t)ustart[e] + r / kTile) * (d / kTile);
+    const uint16_t *xr = x + (int64_t)tok * d;
+    for (int c = 0; c < d; c += 256) {
+        const int i0 = c + 8 * lane;
+        const bool in = i0 < d;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (in) v = __ldg(reinterpret_cast<const uint4 *>(xr + i0));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float f[8], amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+            amax = fmaxf(amax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        uint32_t lo = 0, hi = 0, sb = 127;
+        if (amax > 0.0f) {
+            int se = floor_log2_f32(amax) - 8;
+            se = se < -127 ? -127 : (se > 127 ? 127 : se);
+            sb = (uint32_t)(se + 127);
+            const float sc = pow2_neg(se);
+            lo = f32x2_to_e4m3x2(f[0] * sc, f[1] * sc) | f32x2_to_e4m3x2(f[2] * sc, f[3] * sc) << 16;
+            hi = f32x2_to_e4m3x2(f[4] * sc, f[5] * sc) | f32x2_to_e4m3x2(f[6] * sc, f[7] * sc) << 16;
+        }
+        if (in) {
+            *reinterpret_cast<uint2 *>(x8 + (int64_t)row * d + i0) = make_uint2(lo, hi);
+            if ((lane & 3) == 0) {
+                const int b = i0 / 32;
+                xsf[(atom0 + b / 4) * 512 + sf_atom_byte(r % kTile, b % 4)] = (uint8_t)sb;
+            }
+        }
+    }
+}
+
+int tc_num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+cudaError_t tc_set_attrs() {
+    static bool done[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (done[dev]) return cudaSuccess;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(tc_ffn_kernel<kModeGU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)))
+        return e;
+    if ((e = cudaFuncSetAttribute(tc_ffn_kernel<kModeDN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)))
+        return e;
+    done[dev] = true;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool tc_path_applies(const moe_dims &d) {
+    return d.wfmt == MOE_W_MXFP4 && d.act == MOE_A_MXFP8 && d.d_model % kTile == 0 && d.d_ff % kTile == 0 &&
+           d.E <= kTcMaxE && d.T >= 1;
+}
+
+// Routed expert FFN (w4a8, MXFP4 weights) on the tensor cores: plan, gather +
+// quantise, gate/up GEMM with SwiGLU and MXFP8 requantisation, down GEMM.
+cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
+                          const int32_t *perm, float *out_rows, uint8_t *ws, const WsLayout &L, cudaStream_t s) {
+    const int S = d.T * d.k;
+    if (S == 0) return cudaSuccess;
+    cudaError_t e = tc_set_attrs();
+    if (e != cudaSuccess) return e;
+    const Mxfp4Layout L1 = mxfp4_layout(d, MOE_MAT_W1), L2 = mxfp4_layout(d, MOE_MAT_W2);
+    const uint8_t *p1 = static_cast<const uint8_t *>(w.w1), *p3 = static_cast<const uint8_t *>(w.w3),
+                  *p2 = static_cast<const uint8_t *>(w.w2);
+    int32_t *ustart = reinterpret_cast<int32_t *>(ws + L.ustart);
+    uint8_t *gx8 = ws + L.gx8, *gxsf = ws + L.gxsf, *h8 = ws + L.h8, *hsf = ws + L.ghsf;
+
+    TcArgs g;
+    memset(&g, 0, sizeof g);
+    const uint64_t r13 = (uint64_t)d.E * d.d_ff, r2 = (uint64_t)d.E * d.d_model;
+    bool ok = make_tile_map_e2m1(&g.wa, p1 + L1.codes, r13, d.d_model, kTile) &&
+              make_tile_map_e2m1(&g.wb, p3 + L1.codes, r13, d.d_model, kTile) &&
+              make_tile_map_u8(&g.act, gx8, S, d.d_model, kTile);
+    TcArgs dn;
+    memset(&dn, 0, sizeof dn);
+    ok = ok && make_tile_map_e2m1(&dn.wa, p2 + L2.codes, r2, d.d_ff, kTile) &&
+         make_tile_map_u8(&dn.act, h8, S, d.d_ff, kTile);
+    if (!ok) return cudaErrorInvalidValue;
+    g.sfa = p1 + L1.stile; g.sfb = p3 + L1.stile; g.sfact = gxsf;
+    g.offsets = offsets; g.ustart = ustart; g.E = d.E; g.Nw = d.d_ff; g.K = d.d_model;
+    g.h8 = h8; g.hsf = hsf; g.err = device_error_word();
+    dn.sfa = p2 + L2.stile; dn.sfact = hsf;
+    dn.offsets = offsets; dn.ustart = ustart; dn.E = d.E; dn.Nw = d.d_model; dn.K = d.d_ff;
+    dn.out = out_rows; dn.err = g.err;
+
+    tc_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, ustart);
+    tc_gather_quant_kernel<<<(S + 7) / 8, 256, 0, s>>>(x, offsets, perm, ustart, S, d.E, d.k, d.d_model, gx8, gxsf);
+    const int grid = tc_num_sms();
+    tc_ffn_kernel<kModeGU><<<grid, kTcThreads, kTcSmemBytes, s>>>(g);
+    tc_ffn_kernel<kModeDN><<<grid, kTcThreads, kTcSmemBytes, s>>>(dn);
+    count_launches(4);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

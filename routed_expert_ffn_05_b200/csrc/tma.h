@@ -22,4 +22,15 @@ bool make_chunked_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_
 bool make_plain_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_bytes,
                     uint32_t box_rows);
 
+// Operand tiles for the tensor-core GEMMs: a row-major matrix [rows][K]
+// seen in boxes of 128 K-elements x box_rows rows, 128-byte swizzled (rows of
+// 128 bytes in shared memory, the K-major layout tcgen05.mma reads).
+// u8: one byte per element (E4M3 codes). Base 16-byte aligned, row bytes a
+// multiple of 16.
+bool make_tile_map_u8(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows);
+// e2m1: packed E2M1 codes (two per byte, element 2i in the low nibble),
+// expanded in shared memory to one byte per element (16 codes in the first 8
+// bytes of every 16). Base 32-byte aligned, K a multiple of 128.
+bool make_tile_map_e2m1(CUtensorMap *map, const void *base, uint64_t rows, uint64_t K, uint32_t box_rows);
+
 }  // namespace moe

@@ -293,6 +293,21 @@ def test_layer_edges(T, k, E):
     assert_rel(host(y), ref, TOL["bf16"], f"T={T} k={k} E={E}")
 
 
+@pytest.mark.parametrize("T,k,E", [(1, 1, 8), (37, 2, 8), (300, 3, 16), (260, 4, 4)])
+def test_expert_ffn_w4a8_every_row(T, k, E):
+    """w4a8 expert FFN, every row against the oracle: a single token, ragged
+    token tiles (not multiples of 16), experts with several 128-token tiles and
+    an expert taking every token."""
+    cfg = synth.LayerConfig("w4a8", T=T, d=256, F=512, E=E, k=k, act="mxfp8")
+    c = Case(cfg, experts="all")
+    _, offsets_r, perm_r, _ = oracle.permute(c.ora_idx, cfg.E)
+    out = torch.full((T * k, cfg.d), float("nan"), dtype=torch.float32, device=DEV)
+    M.moe_expert_ffn(c.dims, c.weights, c.x_d, dev(offsets_r), dev(perm_r), out, c.ws)
+    assert M.moe_get_device_error() == 0
+    ref = oracle.expert_ffn_rows(c.ora, c.x, offsets_r, perm_r, 0, T * k)
+    assert_rel(host(out), ref, TOL["mxfp8"], f"w4a8 T={T} k={k} E={E}")
+
+
 def test_identical_tokens_identical_outputs():
     cfg = synth.LayerConfig("dup", T=6, d=256, F=512, E=8, k=2)
     c = Case(cfg, experts="all")
