@@ -10,6 +10,7 @@ timed events. Other configurations are measured in the same run and reported
 under "breakdown".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config decode|prefill|hash|q2k|tiny] [--T T] [--E E]
 
 With N > 1 (torchrun) every rank runs an independent replica on its own
 batches (the path partitions by token batch; no data-path collective) and the
@@ -303,14 +304,32 @@ def oracle_sample(cfg, T, n_tokens, min_seconds, seed=0, batch=0):
 
 # ---- main -------------------------------------------------------------------------
 
+def workload_desc(cfg):
+    fmt = "Q2_K" if cfg.wfmt == "q2k" else "MXFP4"
+    route = "hash (SplitMix64 of the token id)" if cfg.route == "hash" else f"top-{cfg.k} softmax"
+    if cfg.zipf_s:
+        route += f", Zipf({cfg.zipf_s}) router bias"
+    act = "MXFP8 activations (w4a8)" if cfg.act == "mxfp8" else "bf16 activations"
+    sh = f", bf16 shared expert d_ff {cfg.Fs}" if cfg.Fs else ""
+    return (f"{cfg.name} layer T={cfg.T}: d_model {cfg.d}, d_ff {cfg.F}, {cfg.E} {fmt} routed experts, "
+            f"{route} routing, {act}{sh}")
+
+
+def expert_flops(cfg, T):
+    """Useful expert-FFN multiply-adds x 2 of one layer call (routed + shared)."""
+    return 2 * T * cfg.k * 3 * cfg.d * cfg.F + 2 * T * 3 * cfg.d * cfg.Fs
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--T", type=int, default=8)
-    ap.add_argument("--E", type=int, default=256, help="routed experts (smaller only for profiling captures)")
+    ap.add_argument("--config", default="decode", choices=["decode", "prefill", "hash", "q2k", "tiny"],
+                    help="timed workload (default: the decode layer)")
+    ap.add_argument("--T", type=int, default=None, help="tokens per step (default: the config's)")
+    ap.add_argument("--E", type=int, default=None, help="routed experts (smaller only for profiling captures)")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -320,27 +339,31 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     from dataclasses import replace
-    cfg = replace(synth.CONFIGS["decode"].with_T(args.T), E=args.E)
-    workload = (f"decode layer T={args.T}: d_model 4096, d_ff 2048, {args.E} MXFP4 routed experts, top-8 softmax "
-                f"routing, bf16 activations, bf16 shared expert d_ff 2048")
+    base_cfg = synth.CONFIGS[args.config]
+    E = args.E if args.E else base_cfg.E
+    T = args.T if args.T else base_cfg.T
+    cfg = replace(base_cfg.with_T(T), E=E)
+    workload = workload_desc(cfg)
+    n_cpu_tokens = min(T, 8)
 
     if args.impl == "reference":
         if rank != 0:
             return
         per_step = []
         for i in range(args.warmup + args.steps):
-            tps, threads, el, desc = oracle_sample(cfg, args.T, args.T, 0.0, batch=i % NBATCH)
+            tps, threads, el, desc = oracle_sample(cfg, T, n_cpu_tokens, 0.0, batch=i % NBATCH)
             if i >= args.warmup:
-                per_step.append(args.T / tps)
-        ms = 1000 * statistics.mean(per_step)
-        val = args.T / (ms / 1000)
+                per_step.append(n_cpu_tokens / tps)
+        ms = 1000 * statistics.mean(per_step) * T / n_cpu_tokens
+        val = T / (ms / 1000)
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload, "T": args.T},
+            "config": {"workload": workload, "T": T},
             "cpu_baseline": {"kind": "oracle", "value": val, "unit": UNIT, "cores": threads,
-                             "sample": f"each step: oracle layer on the {args.T} tokens of one batch"},
+                             "sample": f"each step: oracle layer on {n_cpu_tokens} of the {T} tokens of one batch, "
+                                       f"scaled to the batch"},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }))
         return
@@ -353,64 +376,94 @@ def main():
     import routed_expert_ffn_05_b200 as M
 
     t0 = time.time()
-    base = DeviceLayer(M, torch, replace(synth.CONFIGS["decode"], E=args.E))
-    log(f"[bench] MXFP4 layer built in {time.time() - t0:.1f}s")
+    if cfg.wfmt == "q2k" or cfg.d != synth.CONFIGS["decode"].d:
+        base = DeviceLayer(M, torch, cfg)
+    else:
+        base = DeviceLayer(M, torch, replace(synth.CONFIGS["decode"], E=E))
+    log(f"[bench] {cfg.wfmt} layer built in {time.time() - t0:.1f}s")
     layer = base.with_weights(cfg)
 
     clocks = Clocks()
     clocks.start()
-    r = measure(M, torch, layer, args.T, args.steps, args.warmup, rank, world)
+    r = measure(M, torch, layer, T, args.steps, args.warmup, rank, world)
     ck = clocks.stop()
     total_s = max_over_ranks(torch, world, sum(r["ms"]) / 1000.0)
-    value = world * args.T * args.steps / total_s
+    value = world * T * args.steps / total_s
     ms_per_step = 1000.0 * total_s / args.steps
 
     if not args.no_e2e:
-        e = measure(M, torch, layer, args.T, args.steps, args.warmup, rank, world, e2e=True)
+        e = measure(M, torch, layer, T, args.steps, args.warmup, rank, world, e2e=True)
         e2e_s = max_over_ranks(torch, world, sum(e["ms"]) / 1000.0)
     else:
         e2e_s = float("nan")
 
-    # roofline of the routed-expert FFN (the dominant stage), per step
+    # roofline of the expert FFN (the dominant stage), per step
     hbm, bf16, src = peaks()
-    xb = torch.from_numpy(synth.make_x(cfg, 0, 1000 * rank).astype(np.int16)).cuda()
-    idx = touched_experts(M, torch, layer, xb, None, args.T)
-    U = len(np.unique(idx))
-    ffn_ms = statistics.mean(r["ffn_ms"][::NBATCH]) if r["ffn_ms"] else float("nan")
-    alg = algorithmic_ffn_bytes(cfg, U)
-    achieved = alg / (ffn_ms / 1000.0) / 1e9
+    ffn_ms = statistics.mean(r["ffn_ms"]) if r["ffn_ms"] else float("nan")
+    if cfg.act == "mxfp8":  # a dense contraction on the FP8 tensor-core rate
+        fl = expert_flops(cfg, T)
+        achieved = fl / (ffn_ms / 1000.0) / 1e12
+        peak = 2.0 * bf16  # E4M3 x E2M1 runs at the FP8 rate: 2x bf16 dense (nominal ratio)
+        roof = {"kernel": "expert FFN: plan + gather/quantise + gate/up GEMM + down GEMM (tcgen05)",
+                "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_source": f"{src} bf16 x 2 (FP8 nominal ratio)",
+                "traffic": None, "algorithmic_flops": fl, "ffn_ms": ffn_ms}
+    else:
+        xb = torch.from_numpy(synth.make_x(cfg, 0, 1000 * rank).astype(np.int16)).cuda()
+        idx = touched_experts(M, torch, layer, xb, None, T)
+        U = len(np.unique(idx))
+        ffn_ms = statistics.mean(r["ffn_ms"][::NBATCH]) if r["ffn_ms"] else float("nan")
+        alg = algorithmic_ffn_bytes(cfg, U)
+        achieved = alg / (ffn_ms / 1000.0) / 1e9
+        roof = {"kernel": "expert FFN: routed + shared", "bound": "hbm",
+                "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_source": src, "traffic": None,
+                "algorithmic_bytes": alg, "experts_touched": U, "ffn_ms": ffn_ms}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "mxfp4 x bf16 -> fp32", "data": "synthetic",
-        "config": {"workload": workload, "T": args.T, "batches": NBATCH,
+        "vs_baseline": None,
+        "dtype": ("mxfp4 x mxfp8 -> fp32" if cfg.act == "mxfp8" else
+                  ("q2k x bf16 -> fp32" if cfg.wfmt == "q2k" else "mxfp4 x bf16 -> fp32")),
+        "data": "synthetic",
+        "config": {"workload": workload, "T": T, "batches": NBATCH,
                    "l2": "flushed between steps (256 MB write), flush outside the timed events",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "roofline": {"kernel": "expert FFN: routed + shared (gate/up + down kernels)", "bound": "hbm",
-                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_source": src, "traffic": None,
-                     "algorithmic_bytes": alg, "experts_touched": U, "ffn_ms": ffn_ms},
-        "e2e": {"value": world * args.T * args.steps / e2e_s, "unit": UNIT,
-                "h2d_bytes_per_step": args.T * cfg.d * 2, "d2h_bytes_per_step": args.T * cfg.d * 4},
+        "roofline": roof,
+        "e2e": {"value": world * T * args.steps / e2e_s, "unit": UNIT,
+                "h2d_bytes_per_step": T * cfg.d * 2 + (T * 4 if cfg.route == "hash" else 0),
+                "d2h_bytes_per_step": T * cfg.d * 4},
         "gpu_launches": r["launches"], "gpu_launches_per_step": r["launches"] / args.steps,
         "clocks": ck,
     }
 
     if not args.no_breakdown and rank == 0:
         bd = {}
-        for T in (1, 2, 4, 8):
-            rr = measure(M, torch, base.with_weights(cfg.with_T(T)), T, 20, 3, rank, 1)
-            bd[f"decode_T{T}"] = {"tokens_per_s": T / (statistics.mean(rr["ms"]) / 1000),
-                                  "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
-        for name in ("prefill", "hash"):
-            c = replace(synth.CONFIGS[name], E=args.E)
-            rr = measure(M, torch, base.with_weights(c), c.T, 3, 3, rank, 1, batches=2)
-            bd[name] = {"T": c.T, "tokens_per_s": c.T / (statistics.mean(rr["ms"]) / 1000),
-                        "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
+        if cfg.wfmt == "mxfp4" and cfg.d == synth.CONFIGS["decode"].d:
+            dec = replace(synth.CONFIGS["decode"], E=E)
+            for Tb in (1, 2, 4, 8):
+                rr = measure(M, torch, base.with_weights(dec.with_T(Tb)), Tb, 20, 3, rank, 1)
+                bd[f"decode_T{Tb}"] = {"tokens_per_s": Tb / (statistics.mean(rr["ms"]) / 1000),
+                                       "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
+            for name in ("prefill", "hash"):
+                c = replace(synth.CONFIGS[name], E=E)
+                rr = measure(M, torch, base.with_weights(c), c.T, 3, 3, rank, 1, batches=2)
+                fl = expert_flops(c, c.T)
+                bd[name] = {"T": c.T, "tokens_per_s": c.T / (statistics.mean(rr["ms"]) / 1000),
+                            "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"]),
+                            "ffn_tflops": fl / (statistics.mean(rr["ffn_ms"]) / 1000) / 1e12}
+            del base
+            torch.cuda.empty_cache()
+            q2 = DeviceLayer(M, torch, replace(synth.CONFIGS["q2k"], E=E))
+            for Tb in (1, 8):
+                rr = measure(M, torch, q2.with_weights(replace(synth.CONFIGS["q2k"], E=E).with_T(Tb)), Tb, 20, 3,
+                             rank, 1)
+                bd[f"q2k_T{Tb}"] = {"tokens_per_s": Tb / (statistics.mean(rr["ms"]) / 1000),
+                                    "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
         line["breakdown"] = bd
 
     if not args.no_cpu and world == 1 and rank == 0:
-        tps, threads, el, desc = oracle_sample(cfg, args.T, args.T, 10.0)
+        tps, threads, el, desc = oracle_sample(cfg, T, n_cpu_tokens, 10.0)
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": desc, "seconds": el}
     if rank == 0:

@@ -48,6 +48,106 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t *__re
     }
 }
 
+// Batch router: a CTA covers 32 tokens x 16 experts; warp w takes 8 tokens x 8
+// experts and lane c the chunk c of every one of its 64 dot products, so each
+// (token, expert) still runs the fixed order above (fma chain per chunk, then
+// the butterfly). Operands are staged per 8-element step of all 32 chunks, as
+// fp32, in [row][half][chunk][4] order: lane c reads 16 contiguous bytes, so a
+// warp's loads hit distinct banks. Requires d % 256 == 0.
+constexpr int kRtT = 32, kRtE = 16;
+constexpr int kRtXs = kRtT * 2 * 32 * 4, kRtWs = kRtE * 2 * 32 * 4;  // floats per buffer
+constexpr int kRtSmem = 2 * (kRtXs + kRtWs) * 4;
+
+__global__ void __launch_bounds__(256, 1) router_tiled_kernel(const uint16_t *__restrict__ x,
+                                                              const uint16_t *__restrict__ wr,
+                                                              const float *__restrict__ bias, int T, int d,
+                                                              int E, float *__restrict__ logits) {
+    extern __shared__ float4 rt_smem[];
+    float *xs = reinterpret_cast<float *>(rt_smem), *ws = xs + 2 * kRtXs;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t_base = blockIdx.y * kRtT, e_base = blockIdx.x * kRtE;
+    const int chunk = d / 32, steps = chunk / 8;
+    // staging: 32 x-rows and 16 w-rows, 32 chunks each, 8 bf16 per (row, chunk)
+    auto load = [&](int st, uint4 (&v)[6]) {
+#pragma unroll
+        for (int q = 0; q < 6; ++q) {
+            const int i = threadIdx.x + 256 * q;  // (row, chunk): rows 0..31 x, 32..47 w
+            const int row = i >> 5, c = i & 31;
+            const bool isx = row < kRtT;
+            const int g = isx ? t_base + row : e_base + row - kRtT;
+            const bool in = g < (isx ? T : E);
+            const uint16_t *src = (isx ? x : wr) + (int64_t)g * d + c * chunk + 8 * st;
+            v[q] = in ? __ldg(reinterpret_cast<const uint4 *>(src)) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    auto store = [&](int buf, const uint4 (&v)[6]) {
+#pragma unroll
+        for (int q = 0; q < 6; ++q) {
+            const int i = threadIdx.x + 256 * q;
+            const int row = i >> 5, c = i & 31;
+            float *dst = row < kRtT ? xs + buf * kRtXs + (row * 2) * 128 + c * 4
+                                    : ws + buf * kRtWs + ((row - kRtT) * 2) * 128 + c * 4;
+            const uint32_t a[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+            reinterpret_cast<float4 *>(dst)[0] = make_float4(__uint_as_float(a[0] << 16), __uint_as_float(a[0] & 0xFFFF0000u),
+                                                             __uint_as_float(a[1] << 16), __uint_as_float(a[1] & 0xFFFF0000u));
+            reinterpret_cast<float4 *>(dst + 128)[0] = make_float4(__uint_as_float(a[2] << 16), __uint_as_float(a[2] & 0xFFFF0000u),
+                                                                   __uint_as_float(a[3] << 16), __uint_as_float(a[3] & 0xFFFF0000u));
+        }
+    };
+    const int tw = (warp >> 1) * 8, ew = (warp & 1) * 8;  // this warp's 8 tokens, 8 experts
+    float acc[8][8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+    uint4 v[6];
+    load(0, v);
+    store(0, v);
+    __syncthreads();
+    for (int st = 0; st < steps; ++st) {
+        const int buf = st & 1;
+        if (st + 1 < steps) load(st + 1, v);
+        const float *xb = xs + buf * kRtXs, *wb = ws + buf * kRtWs;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float4 xv[8], wv[8];
+#pragma unroll
+            for (int a = 0; a < 8; ++a) xv[a] = reinterpret_cast<const float4 *>(xb + ((tw + a) * 2 + h) * 128)[lane];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) wv[b] = reinterpret_cast<const float4 *>(wb + ((ew + b) * 2 + h) * 128)[lane];
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 8; ++b) {
+                    acc[a][b] = __fmaf_rn(xv[a].x, wv[b].x, acc[a][b]);
+                    acc[a][b] = __fmaf_rn(xv[a].y, wv[b].y, acc[a][b]);
+                    acc[a][b] = __fmaf_rn(xv[a].z, wv[b].z, acc[a][b]);
+                    acc[a][b] = __fmaf_rn(xv[a].w, wv[b].w, acc[a][b]);
+                }
+        }
+        if (st + 1 < steps) store(buf ^ 1, v);
+        __syncthreads();
+    }
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            float p = acc[a][b];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
+            acc[a][b] = p;
+        }
+    // every lane holds every sum now; lane (8a + b) % 32 writes (tw + a, ew + b)
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const int t = t_base + tw + a, e = e_base + ew + b;
+            if (lane == ((8 * a + b) & 31) && t < T && e < E)
+                logits[(int64_t)t * E + e] = bias ? __fadd_rn(acc[a][b], bias[e]) : acc[a][b];
+        }
+}
+
 // a ranks before b: larger logit first, NaN after every number, ties (and
 // +0 == -0) by the lower index.
 __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
@@ -135,9 +235,22 @@ cudaError_t launch_route(const moe_dims &d, const uint16_t *x, const moe_weights
         count_launches(1);
         return cudaGetLastError();
     }
-    const int ey = ceil_div(d.E, 8);
-    router_logits_kernel<<<dim3(d.T, ey), 256, d.d_model * 2, s>>>(x, wt.w_router, wt.router_bias, d.T,
-                                                                      d.d_model, d.E, logits);
+    if (d.T >= kRtT && d.d_model % 256 == 0) {
+        static bool attr_set[64] = {false};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(router_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRtSmem);
+            if (e != cudaSuccess) return e;
+            attr_set[dev] = true;
+        }
+        router_tiled_kernel<<<dim3(ceil_div(d.E, kRtE), ceil_div(d.T, kRtT)), 256, kRtSmem, s>>>(
+            x, wt.w_router, wt.router_bias, d.T, d.d_model, d.E, logits);
+    } else {
+        const int ey = ceil_div(d.E, 8);
+        router_logits_kernel<<<dim3(d.T, ey), 256, d.d_model * 2, s>>>(x, wt.w_router, wt.router_bias, d.T,
+                                                                          d.d_model, d.E, logits);
+    }
     topk_softmax_kernel<<<ceil_div(d.T, 8), 256, 0, s>>>(logits, d.T, d.E, d.k, idx, w);
     count_launches(2);
     return cudaGetLastError();
