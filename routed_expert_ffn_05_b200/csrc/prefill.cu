@@ -236,55 +236,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                 break;
             }
             tc_fence_after();
-            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-                if (c0 >= wk.nvalid) break;
-                uint32_t g[32];
-                tmem_ld32(lane_base + c0, g);
-                if (GU) {
-                    uint32_t u[32];
-                    tmem_ld32(lane_base + 128 + c0, u);
-                    tmem_wait_ld();
-                    const int fcol = wk.f * kTile + 32 * q + lane;  // this lane's h column
-                    const int64_t atom = (((int64_t)s.ustart[wk.e] + wk.j) * (a.Nw / kTile) + wk.f) * 512;
+            // Pull this warp's columns out of TMEM (gate/up: h = silu(g) u right
+            // away), then hand the accumulator back before the slow part, so the
+            // next tile's MMAs overlap the requantisation and the stores.
+            const int c0 = 64 * half;
+            const int nc = max(0, min(64, wk.nvalid - c0));  // this warp's valid columns
+            float v[64];
+            if (nc > 0) {
+                uint32_t r[32];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        float hv[2];
-                        int se[2];
+                for (int c = 0; c < 2; ++c) {
+                    if (c * 32 < nc) {  // warp-uniform
+                        tmem_ld32(lane_base + c0 + 32 * c, r);
+                        if (GU) {
+                            uint32_t u[32];
+                            tmem_ld32(lane_base + 128 + c0 + 32 * c, u);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            const float gv = __uint_as_float(g[i + p]);
-                            hv[p] = silu_f32(gv) * __uint_as_float(u[i + p]);
-                            const uint32_t amax = warp_max_u32(__float_as_uint(hv[p]) & 0x7FFFFFFFu);
-                            if (amax == 0u) {
-                                se[p] = 0;
-                                hv[p] = 0.0f;
-                            } else {
-                                int e8 = floor_log2_f32(__uint_as_float(amax)) - 8;
-                                se[p] = e8 < -127 ? -127 : (e8 > 127 ? 127 : e8);
-                                hv[p] *= pow2_neg(se[p]);
+                            for (int i = 0; i < 32; ++i) {
+                                const float gv = __uint_as_float(r[i]);
+                                v[32 * c + i] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[i]);
                             }
-                        }
-                        const uint32_t codes = f32x2_to_e4m3x2(hv[0], hv[1]);
+                        } else {
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            const int t = c0 + i + p;
-                            if (t < wk.nvalid) {
-                                a.h8[(int64_t)(wk.row0 + t) * a.Nw + fcol] = (uint8_t)(codes >> (8 * p));
-                                if (lane == 0) a.hsf[atom + sf_atom_byte(t, q)] = (uint8_t)(se[p] + 127);
-                            }
+                            for (int i = 0; i < 32; ++i) v[32 * c + i] = __uint_as_float(r[i]);
                         }
                     }
-                } else {
-                    tmem_wait_ld();
-                    float *orow = a.out + (int64_t)wk.row0 * a.Nw + wk.f * kTile + 32 * q + lane;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c0 + i < wk.nvalid) orow[(int64_t)(c0 + i) * a.Nw] = __uint_as_float(g[i]);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.acc_empty);
+            if (GU) {
+                // MXFP8 along F: the block of 32 is this warp's 32 lanes
+                const int fcol = wk.f * kTile + 32 * q + lane;  // this lane's h column
+                const int64_t atom = (((int64_t)s.ustart[wk.e] + wk.j) * (a.Nw / kTile) + wk.f) * 512;
+                uint8_t *hrow = a.h8 + (int64_t)(wk.row0 + c0) * a.Nw + fcol;
+#pragma unroll
+                for (int i = 0; i < 64; i += 2) {
+                    if (i >= nc) break;  // warp-uniform
+                    float hv[2];
+                    int se[2];
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        hv[p] = v[i + p];
+                        const uint32_t amax = warp_max_u32(__float_as_uint(hv[p]) & 0x7FFFFFFFu);
+                        if (amax == 0u) {
+                            se[p] = 0;
+                            hv[p] = 0.0f;
+                        } else {
+                            const int e8 = floor_log2_f32(__uint_as_float(amax)) - 8;
+                            se[p] = e8 < -127 ? -127 : (e8 > 127 ? 127 : e8);
+                            hv[p] *= pow2_neg(se[p]);
+                        }
+                    }
+                    const uint32_t codes = f32x2_to_e4m3x2(hv[0], hv[1]);
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        if (i + p < nc) {
+                            hrow[(int64_t)(i + p) * a.Nw] = (uint8_t)(codes >> (8 * p));
+                            if (lane == 0) a.hsf[atom + sf_atom_byte(c0 + i + p, q)] = (uint8_t)(se[p] + 127);
+                        }
+                    }
+                }
+            } else {
+                float *orow = a.out + (int64_t)(wk.row0 + c0) * a.Nw + wk.f * kTile + 32 * q + lane;
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if (i < nc) orow[(int64_t)i * a.Nw] = v[i];
+            }
         }
     }
     tc_fence_before();
