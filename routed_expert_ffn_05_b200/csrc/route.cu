@@ -14,6 +14,10 @@
 #include "kernels.h"
 
 namespace moe {
+__device__ __forceinline__ uint32_t smem_u32_rt(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+}  // namespace moe
+
+namespace moe {
 
 // Decode-sized router: one warp per (token, expert), the token's x row staged
 // once per block in shared memory.
@@ -48,102 +52,105 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t *__re
     }
 }
 
-// Batch router: a CTA covers 32 tokens x 16 experts; warp w takes 8 tokens x 8
-// experts and lane c the chunk c of every one of its 64 dot products, so each
+// Batch router: a CTA covers 32 tokens x 32 experts; warp w takes 8 tokens x
+// 16 experts and lane c the chunk c of each of its 128 dot products, so every
 // (token, expert) still runs the fixed order above (fma chain per chunk, then
-// the butterfly). Operands are staged per 8-element step of all 32 chunks, as
-// fp32, in [row][half][chunk][4] order: lane c reads 16 contiguous bytes, so a
-// warp's loads hit distinct banks. Requires d % 256 == 0.
-constexpr int kRtT = 32, kRtE = 16;
-constexpr int kRtXs = kRtT * 2 * 32 * 4, kRtWs = kRtE * 2 * 32 * 4;  // floats per buffer
-constexpr int kRtSmem = 2 * (kRtXs + kRtWs) * 4;
+// the butterfly). Operands are copied as bf16 with cp.async, 8 elements of
+// every chunk per step, in [row][chunk][8] order (lane c reads 8 contiguous
+// bytes at a 16-byte stride), three steps in flight; values widen to fp32 on
+// read. Requires d % 256 == 0.
+constexpr int kRtT = 32, kRtE = 32, kRtStages = 3;
+constexpr int kRtRowBytes = 32 * 16;                          // one row: 32 chunks x 8 bf16
+constexpr int kRtStageBytes = (kRtT + kRtE) * kRtRowBytes;    // 32 KB
+constexpr int kRtSmem = kRtStages * kRtStageBytes;
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool in) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32_rt(dst)), "l"(src), "r"(in ? 16 : 0)
+                 : "memory");
+}
 
 __global__ void __launch_bounds__(256, 1) router_tiled_kernel(const uint16_t *__restrict__ x,
                                                               const uint16_t *__restrict__ wr,
                                                               const float *__restrict__ bias, int T, int d,
                                                               int E, float *__restrict__ logits) {
-    extern __shared__ float4 rt_smem[];
-    float *xs = reinterpret_cast<float *>(rt_smem), *ws = xs + 2 * kRtXs;
+    extern __shared__ uint4 rt_smem[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(rt_smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t_base = blockIdx.y * kRtT, e_base = blockIdx.x * kRtE;
     const int chunk = d / 32, steps = chunk / 8;
-    // staging: 32 x-rows and 16 w-rows, 32 chunks each, 8 bf16 per (row, chunk)
-    auto load = [&](int st, uint4 (&v)[6]) {
+    // step st: rows 0..31 x, 32..63 w; 8 bf16 of every chunk; zero-filled past T / E
+    auto issue = [&](int st) {
+        uint8_t *dst0 = sm + (st % kRtStages) * kRtStageBytes;
 #pragma unroll
-        for (int q = 0; q < 6; ++q) {
-            const int i = threadIdx.x + 256 * q;  // (row, chunk): rows 0..31 x, 32..47 w
+        for (int q = 0; q < 8; ++q) {
+            const int i = threadIdx.x + 256 * q;
             const int row = i >> 5, c = i & 31;
             const bool isx = row < kRtT;
             const int g = isx ? t_base + row : e_base + row - kRtT;
             const bool in = g < (isx ? T : E);
-            const uint16_t *src = (isx ? x : wr) + (int64_t)g * d + c * chunk + 8 * st;
-            v[q] = in ? __ldg(reinterpret_cast<const uint4 *>(src)) : make_uint4(0, 0, 0, 0);
+            const uint16_t *src = (isx ? x : wr) + (int64_t)(in ? g : 0) * d + c * chunk + 8 * st;
+            cp_async16(dst0 + row * kRtRowBytes + c * 16, src, in);
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    auto store = [&](int buf, const uint4 (&v)[6]) {
-#pragma unroll
-        for (int q = 0; q < 6; ++q) {
-            const int i = threadIdx.x + 256 * q;
-            const int row = i >> 5, c = i & 31;
-            float *dst = row < kRtT ? xs + buf * kRtXs + (row * 2) * 128 + c * 4
-                                    : ws + buf * kRtWs + ((row - kRtT) * 2) * 128 + c * 4;
-            const uint32_t a[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-            reinterpret_cast<float4 *>(dst)[0] = make_float4(__uint_as_float(a[0] << 16), __uint_as_float(a[0] & 0xFFFF0000u),
-                                                             __uint_as_float(a[1] << 16), __uint_as_float(a[1] & 0xFFFF0000u));
-            reinterpret_cast<float4 *>(dst + 128)[0] = make_float4(__uint_as_float(a[2] << 16), __uint_as_float(a[2] & 0xFFFF0000u),
-                                                                   __uint_as_float(a[3] << 16), __uint_as_float(a[3] & 0xFFFF0000u));
-        }
-    };
-    const int tw = (warp >> 1) * 8, ew = (warp & 1) * 8;  // this warp's 8 tokens, 8 experts
-    float acc[8][8];
+    const int tw = (warp >> 1) * 8, ew = kRtT + (warp & 1) * 16;  // this warp's rows (x, w)
+    float acc[8][16];
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
-    uint4 v[6];
-    load(0, v);
-    store(0, v);
-    __syncthreads();
+        for (int b = 0; b < 16; ++b) acc[a][b] = 0.0f;
+    for (int st = 0; st < kRtStages - 1; ++st) {
+        if (st < steps) issue(st);
+        else asm volatile("cp.async.commit_group;" ::: "memory");
+    }
     for (int st = 0; st < steps; ++st) {
-        const int buf = st & 1;
-        if (st + 1 < steps) load(st + 1, v);
-        const float *xb = xs + buf * kRtXs, *wb = ws + buf * kRtWs;
+        asm volatile("cp.async.wait_group %0;" ::"n"(kRtStages - 2) : "memory");
+        __syncthreads();
+        if (st + kRtStages - 1 < steps) issue(st + kRtStages - 1);
+        else asm volatile("cp.async.commit_group;" ::: "memory");
+        const uint8_t *b0 = sm + (st % kRtStages) * kRtStageBytes + lane * 16;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            float4 xv[8], wv[8];
+            uint2 xp[8], wp[16];
 #pragma unroll
-            for (int a = 0; a < 8; ++a) xv[a] = reinterpret_cast<const float4 *>(xb + ((tw + a) * 2 + h) * 128)[lane];
+            for (int a = 0; a < 8; ++a) xp[a] = *reinterpret_cast<const uint2 *>(b0 + (tw + a) * kRtRowBytes + 8 * h);
 #pragma unroll
-            for (int b = 0; b < 8; ++b) wv[b] = reinterpret_cast<const float4 *>(wb + ((ew + b) * 2 + h) * 128)[lane];
+            for (int b = 0; b < 16; ++b) wp[b] = *reinterpret_cast<const uint2 *>(b0 + (ew + b) * kRtRowBytes + 8 * h);
 #pragma unroll
-            for (int a = 0; a < 8; ++a)
+            for (int j = 0; j < 4; ++j) {  // element 8 st + 4 h + j of every chunk, ascending
+                float xf[8];
 #pragma unroll
-                for (int b = 0; b < 8; ++b) {
-                    acc[a][b] = __fmaf_rn(xv[a].x, wv[b].x, acc[a][b]);
-                    acc[a][b] = __fmaf_rn(xv[a].y, wv[b].y, acc[a][b]);
-                    acc[a][b] = __fmaf_rn(xv[a].z, wv[b].z, acc[a][b]);
-                    acc[a][b] = __fmaf_rn(xv[a].w, wv[b].w, acc[a][b]);
+                for (int a = 0; a < 8; ++a) {
+                    const uint32_t v = j < 2 ? xp[a].x : xp[a].y;
+                    xf[a] = __uint_as_float((j & 1) ? (v & 0xFFFF0000u) : (v << 16));
                 }
+#pragma unroll
+                for (int b = 0; b < 16; ++b) {
+                    const uint32_t v = j < 2 ? wp[b].x : wp[b].y;
+                    const float wf = __uint_as_float((j & 1) ? (v & 0xFFFF0000u) : (v << 16));
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) acc[a][b] = __fmaf_rn(xf[a], wf, acc[a][b]);
+                }
+            }
         }
-        if (st + 1 < steps) store(buf ^ 1, v);
-        __syncthreads();
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
+        for (int b = 0; b < 16; ++b) {
             float p = acc[a][b];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
             acc[a][b] = p;
         }
-    // every lane holds every sum now; lane (8a + b) % 32 writes (tw + a, ew + b)
+    // every lane holds every sum now; lane (16a + b) % 32 writes (token tw + a, expert b)
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const int t = t_base + tw + a, e = e_base + ew + b;
-            if (lane == ((8 * a + b) & 31) && t < T && e < E)
+        for (int b = 0; b < 16; ++b) {
+            const int t = t_base + tw + a, e = e_base + (warp & 1) * 16 + b;
+            if (lane == ((16 * a + b) & 31) && t < T && e < E)
                 logits[(int64_t)t * E + e] = bias ? __fadd_rn(acc[a][b], bias[e]) : acc[a][b];
         }
 }
