@@ -33,6 +33,8 @@
 // k-slots of both k16 steps.
 #include <string.h>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -47,7 +49,9 @@ constexpr int kEpilogue = kCW + 1;        // warp index of the epilogue warp
 constexpr int kThreads = (kCW + 2) * 32;
 constexpr int kStages = 4;
 constexpr int kStageW = 32768;            // weight tile bytes per stage
-constexpr int kStageS = 2048;             // scale bytes per stage
+constexpr int kStageS = 10240;            // scale / metadata bytes per stage (MXFP4: 2 KB of E8M0;
+                                          // Q2_K: 8 KB of sc|m bytes + 2 KB of (d, dmin))
+constexpr int kQDd = 8192;                // Q2_K: offset of the (d, dmin) pairs in a stage's metadata
 constexpr int kMaxE = 1024;
 constexpr int kD = 4096, kF = 2048;       // the dims this tiling is written for
 constexpr int kGuTiles = kF / 16;         // gate/up tiles per routed expert
@@ -60,9 +64,10 @@ constexpr int kDshTiles = kD / 16;        // shared-expert down tiles
 enum { kGsh = 0, kGrt = 1, kDsh = 2, kDrt = 3 };
 
 struct DecodeArgs {
-    CUtensorMap m1c, m3c, m2c;  // routed codes, chunked + swizzled
-    CUtensorMap m1s, m3s, m2s;  // routed row-major scales
+    CUtensorMap m1c, m3c, m2c;  // routed MXFP4 codes or Q2_K quants, chunked + swizzled
+    CUtensorMap m1s, m3s, m2s;  // routed MXFP4 row-major scales, or Q2_K sc|m bytes (chunked)
     CUtensorMap ms1, ms3, ms2;  // shared expert (bf16), chunked + swizzled
+    CUtensorMap m1d, m3d, m2d;  // Q2_K (d, dmin) pairs, row-major
     int T, E, k, Fs;
     const int32_t *offsets, *perm;
     const uint16_t *x;       // [T][d] bf16
@@ -114,10 +119,15 @@ struct Unit {
 // Shared gate/up units are assigned statically (they need no routing), routed
 // gate/up units through the work queue, and the down units as one contiguous,
 // stage-balanced range per CTA (few expert changes, so few reloads of h).
+// A routed gate/up unit is 16 rows of W1 and W3 over all K: two stages of
+// MXFP4 codes, or one stage of Q2_K quants (half the bytes).
+template <int WF> constexpr int gu_stages() { return WF == MOE_W_Q2K ? 1 : 2; }
+
+template <int WF>
 __device__ __forceinline__ Unit unit_of(int u, int usg, int n_seg, int usd) {
     if (u < usg) return Unit{kGsh, -1, u, 8};
     int r = u - usg;
-    if (r < n_seg * kGuTiles) return Unit{kGrt, r / kGuTiles, r % kGuTiles, 2};
+    if (r < n_seg * kGuTiles) return Unit{kGrt, r / kGuTiles, r % kGuTiles, gu_stages<WF>()};
     r -= n_seg * kGuTiles;
     if (r < usd) return Unit{kDsh, -1, r, 2};
     r -= usd;
@@ -198,7 +208,123 @@ __device__ __forceinline__ float row_scale(uint32_t hm) {  // 2^p with max |h| *
     return ldexpf(1.0f, hm ? floor_log2_f32(__uint_as_float(hm)) - 14 : 0);
 }
 
+// ---- Q2_K ----
+// Quants are stored in lane order (see layout.h): the 32-bit word 4G + q of a
+// super-block holds lane q's quants of sub-blocks 4G .. 4G + 3 as 8 pairs,
+// pair k = 2 (sub-block % 4) + h with its two quants 16 bits apart. MMA k-slots
+// 2q, 2q+1 carry elements 4q, 4q+1 of a 16-element sub-block (h = 0) and
+// k-slots 2q+8, 2q+9 elements 4q+2, 4q+3 (h = 1). Pair k is masked out of the
+// word shifted by 6 (k / 3), at bit 2 (k % 3), so it carries 4^(k % 3) q; an
+// integer multiply by the sub-block scale sc gives sc q 4^(k % 3) <= 720 in
+// each 16-bit half, used directly as an f16 subnormal (value x 2^-24, exact).
+// The activation k-slots of pair k are pre-scaled by 4^-(k % 3).
+template <int K>
+__device__ __forceinline__ uint32_t q2_pair(uint32_t w, uint32_t sc) {
+    return ((w >> (6 * (K / 3))) & (0x00030003u << (2 * (K % 3)))) * sc;
+}
+__host__ __device__ constexpr float q2_pre(int k) { return k % 3 == 0 ? 1.0f : (k % 3 == 1 ? 0.25f : 0.0625f); }
+
+// One super-block (16 sub-blocks of 16) of 16 rows r0 + g, r0 + g + 8 of a
+// Q2_K box (quants: `rows` rows, 128-byte chunks; sc|m: same rows, chunked;
+// dd: row-major, `ddrow` bytes per row) against B (16 sub-blocks) and bm (the
+// sub-block sums as f16 hi + lo parts: bm[0..1] hi, bm[2..3] lo).
+// acc += d (sum_j sc_j q . x) - dmin (sum_j m_j xsum_j).
+__device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, const uint8_t *scm,
+                                               const uint8_t *dd, int rows, int ddrow, int r0, int sb, int g,
+                                               int q, const uint32_t (*B)[4], const uint32_t bm[4]) {
+    const int rg = r0 + g, rh = r0 + g + 8;
+    const uint4 ml = lds128(scm + swz_off((sb * 16) / 128, rows, rg, sb % 8));
+    const uint4 mh = lds128(scm + swz_off((sb * 16) / 128, rows, rh, sb % 8));
+    const uint32_t sl[4] = {ml.x, ml.y, ml.z, ml.w}, sh[4] = {mh.x, mh.y, mh.z, mh.w};
+    float tm[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int G = 0; G < 4; ++G) {
+        const int c = (sb * 64) / 128, u = 4 * (sb & 1) + G;
+        const uint32_t wl = lds32(qs + swz_off(c, rows, rg, u) + 4 * q);
+        const uint32_t wh = lds32(qs + swz_off(c, rows, rh, u) + 4 * q);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t cl = (sl[G] >> (8 * jj)) & 15u, ch = (sh[G] >> (8 * jj)) & 15u;
+            uint32_t a0, a1, a2, a3;
+            switch (jj) {  // pair indices are compile-time constants
+                case 0: a0 = q2_pair<0>(wl, cl); a1 = q2_pair<0>(wh, ch); a2 = q2_pair<1>(wl, cl); a3 = q2_pair<1>(wh, ch); break;
+                case 1: a0 = q2_pair<2>(wl, cl); a1 = q2_pair<2>(wh, ch); a2 = q2_pair<3>(wl, cl); a3 = q2_pair<3>(wh, ch); break;
+                case 2: a0 = q2_pair<4>(wl, cl); a1 = q2_pair<4>(wh, ch); a2 = q2_pair<5>(wl, cl); a3 = q2_pair<5>(wh, ch); break;
+                default: a0 = q2_pair<6>(wl, cl); a1 = q2_pair<6>(wh, ch); a2 = q2_pair<7>(wl, cl); a3 = q2_pair<7>(wh, ch);
+            }
+            const int j = 4 * G + jj;
+            mma_f16_16816(tm, a0, a1, a2, a3, B[j >> 1][2 * (j & 1)], B[j >> 1][2 * (j & 1) + 1]);
+        }
+    }
+    // minimum term: A = m of sub-blocks 2q, 2q+1 (k-slots 2q, 2q+1) and 2q+8, 2q+9
+    auto mpair = [&](uint32_t w) {  // bytes 0, 1 of w -> their high nibbles as an f16 subnormal pair
+        return ((w >> 4) & 0xFu) | ((w << 4) & 0xF0000u);
+    };
+    const int sh16 = 16 * (q & 1);
+    const uint32_t lA = (q < 2 ? ml.x : ml.y) >> sh16, lB = (q < 2 ? ml.z : ml.w) >> sh16;
+    const uint32_t hA = (q < 2 ? mh.x : mh.y) >> sh16, hB = (q < 2 ? mh.z : mh.w) >> sh16;
+    float tn[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t ma0 = mpair(lA), ma1 = mpair(hA), ma2 = mpair(lB), ma3 = mpair(hB);
+    mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[0], bm[1]);
+    mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[2], bm[3]);
+    const uint32_t dl = lds32(dd + rg * ddrow + 4 * sb), dh = lds32(dd + rh * ddrow + 4 * sb);
+    // 2^24 undoes the subnormal encoding; 2^5 the sub-block-sum pre-scale
+    const float d0 = __half2float(__ushort_as_half((uint16_t)(dl & 0xFFFF))) * 16777216.0f;
+    const float m0 = __half2float(__ushort_as_half((uint16_t)(dl >> 16))) * 536870912.0f;
+    const float d1 = __half2float(__ushort_as_half((uint16_t)(dh & 0xFFFF))) * 16777216.0f;
+    const float m1 = __half2float(__ushort_as_half((uint16_t)(dh >> 16))) * 536870912.0f;
+    acc[0] = fmaf(-m0, tn[0], fmaf(d0, tm[0], acc[0]));
+    acc[1] = fmaf(-m0, tn[1], fmaf(d0, tm[1], acc[1]));
+    acc[2] = fmaf(-m1, tn[2], fmaf(d1, tm[2], acc[2]));
+    acc[3] = fmaf(-m1, tn[3], fmaf(d1, tm[3], acc[3]));
+}
+
+// B fragments of `nsb` super-blocks (16 sub-blocks each) of one activation row
+// (bf16, scaled by `inv`): k-slot pre-scale 4^-(k % 3), the elements of lane q
+// as described above; bm gets the sub-block sums (scaled by 2^-5) of
+// sub-blocks 2q, 2q+1, 2q+8, 2q+9 of each super-block, each split into an f16
+// part and the f16 of its remainder (together ~22 bits: the minimum term
+// nearly cancels the main term, so its sums need more than f16).
+template <int NSB, bool CG>
+__device__ __forceinline__ void q2k_load_b(const uint16_t *row, float inv, int q, uint32_t (*B)[4],
+                                           uint32_t (*bm)[4]) {
+#pragma unroll
+    for (int s2 = 0; s2 < NSB; ++s2) {
+        float keep[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint16_t *src = row + 256 * s2 + 16 * j + 4 * q;
+            const uint2 v = CG ? __ldcg(reinterpret_cast<const uint2 *>(src)) : __ldg(reinterpret_cast<const uint2 *>(src));
+            const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xFFFF0000u);
+            const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xFFFF0000u);
+            const int jl = 16 * s2 + j;
+            const float c0 = inv * q2_pre(2 * (j & 3)), c1 = inv * q2_pre(2 * (j & 3) + 1);
+            B[jl >> 1][2 * (jl & 1)] = f32x2_to_f16x2(x0 * c0, x1 * c0);
+            B[jl >> 1][2 * (jl & 1) + 1] = f32x2_to_f16x2(x2 * c1, x3 * c1);
+            float ps = (x0 + x1) + (x2 + x3);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+            if (j < 8 && (j >> 1) == q) keep[j & 1] = ps;
+            if (j >= 8 && ((j - 8) >> 1) == q) keep[2 + (j & 1)] = ps;
+        }
+        const float xs = inv * 0.03125f;
+        float hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float v = keep[i] * xs;
+            hi[i] = __half2float(__float2half_rn(v));
+            lo[i] = v - hi[i];
+        }
+        bm[s2][0] = f32x2_to_f16x2(hi[0], hi[1]);
+        bm[s2][1] = f32x2_to_f16x2(hi[2], hi[3]);
+        bm[s2][2] = f32x2_to_f16x2(lo[0], lo[1]);
+        bm[s2][3] = f32x2_to_f16x2(lo[2], lo[3]);
+    }
+}
+
+template <int WF>
 __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr bool Q2 = WF == MOE_W_Q2K;
     extern __shared__ uint8_t smem_raw[];
     Smem &s = smem_ref(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -241,27 +367,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                         tma_load_3d(w + 16384, &a.ms3, 0, 16 * un.tile, 8 * c, bar);
                         break;
                     case kGrt:
-                        arm(s, slot, u, c, 2 * 16384 + 2 * 1024);
-                        tma_load_3d(w, &a.m1c, 0, row0, 8 * c, bar);
-                        tma_load_3d(w + 16384, &a.m3c, 0, row0, 8 * c, bar);
-                        tma_load_2d(s.s[slot], &a.m1s, 64 * c, row0, bar);
-                        tma_load_2d(s.s[slot] + 1024, &a.m3s, 64 * c, row0, bar);
+                        if (Q2) {  // quants, sc|m bytes and (d, dmin) of 16 rows over all K
+                            arm(s, slot, u, c, 2 * 16384 + 2 * 4096 + 2 * 1024);
+                            tma_load_3d(w, &a.m1c, 0, row0, 0, bar);
+                            tma_load_3d(w + 16384, &a.m3c, 0, row0, 0, bar);
+                            tma_load_3d(s.s[slot], &a.m1s, 0, row0, 0, bar);
+                            tma_load_3d(s.s[slot] + 4096, &a.m3s, 0, row0, 0, bar);
+                            tma_load_2d(s.s[slot] + kQDd, &a.m1d, 0, row0, bar);
+                            tma_load_2d(s.s[slot] + kQDd + 1024, &a.m3d, 0, row0, bar);
+                        } else {
+                            arm(s, slot, u, c, 2 * 16384 + 2 * 1024);
+                            tma_load_3d(w, &a.m1c, 0, row0, 8 * c, bar);
+                            tma_load_3d(w + 16384, &a.m3c, 0, row0, 8 * c, bar);
+                            tma_load_2d(s.s[slot], &a.m1s, 64 * c, row0, bar);
+                            tma_load_2d(s.s[slot] + 1024, &a.m3s, 64 * c, row0, bar);
+                        }
                         break;
                     case kDsh:
                         arm(s, slot, u, c, 32768);
                         tma_load_3d(w, &a.ms2, 0, 16 * un.tile, 16 * c, bar);
                         break;
                     default:
-                        arm(s, slot, u, c, 32768 + 2048);
-                        tma_load_3d(w, &a.m2c, 0, row0, 0, bar);
-                        tma_load_2d(s.s[slot], &a.m2s, 0, row0, bar);
+                        if (Q2) {  // 32 rows of W2 over all K
+                            arm(s, slot, u, c, 16384 + 4096 + 1024);
+                            tma_load_3d(w, &a.m2c, 0, row0, 0, bar);
+                            tma_load_3d(s.s[slot], &a.m2s, 0, row0, 0, bar);
+                            tma_load_2d(s.s[slot] + kQDd, &a.m2d, 0, row0, bar);
+                        } else {
+                            arm(s, slot, u, c, 32768 + 2048);
+                            tma_load_3d(w, &a.m2c, 0, row0, 0, bar);
+                            tma_load_2d(s.s[slot], &a.m2s, 0, row0, bar);
+                        }
                 }
             }
         };
         if (lane == 0) {
             prefetch_tensormap(&a.m1c);
             prefetch_tensormap(&a.m2c);
-            for (int u = blockIdx.x; u < usg && !s.abort; u += gridDim.x) issue(u, unit_of(u, usg, 0, 0));
+            for (int u = blockIdx.x; u < usg && !s.abort; u += gridDim.x) issue(u, unit_of<WF>(u, usg, 0, 0));
         }
         __syncwarp();
         grid_dep_wait();  // routing results and zeroed counters from here on
@@ -283,21 +426,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         // queue alone when the static split would not be monotonic.
         const int R = n * kGuTiles;
         int Rs = R - R / 4;
-        const long long tot = 8ll * usg + 2ll * Rs;
+        constexpr int kGuSt = gu_stages<WF>();
+        const long long tot = 8ll * usg + (long long)kGuSt * Rs;
         if (usg > (int)gridDim.x || tot < 8ll * gridDim.x) Rs = 0;
         auto rstart = [&](int b) {
             const long long st = tot * b / gridDim.x - 8ll * min(b, usg);
-            return (int)min((long long)Rs, max(0ll, (st + 1) / 2));
+            return (int)min((long long)Rs, max(0ll, (st + kGuSt - 1) / kGuSt));
         };
         const int rs0 = Rs ? rstart(blockIdx.x) : 0, rs1 = Rs ? rstart(blockIdx.x + 1) : 0;
-        for (int u = usg + rs0; u < usg + rs1 && !s.abort; ++u) issue(u, unit_of(u, usg, n, usd));
+        for (int u = usg + rs0; u < usg + rs1 && !s.abort; ++u) issue(u, unit_of<WF>(u, usg, n, usd));
         constexpr int kGrab = 2;
         int next = usg + Rs + (int)atomicAdd(a.counters, (uint32_t)kGrab);
         while (!s.abort) {  // the next chunk is fetched one chunk ahead
             const int u0 = next;
             if (u0 >= gu_end) break;
             next = usg + Rs + (int)atomicAdd(a.counters, (uint32_t)kGrab);
-            for (int u = u0; u < min(u0 + kGrab, gu_end) && !s.abort; ++u) issue(u, unit_of(u, usg, n, usd));
+            for (int u = u0; u < min(u0 + kGrab, gu_end) && !s.abort; ++u) issue(u, unit_of<WF>(u, usg, n, usd));
         }
         // this CTA's contiguous share of the down units (shared tiles cost 2 stages)
         const long long cost = 2ll * usd + (long long)n * kDnTiles;
@@ -305,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             return gu_end + (cst <= 2ll * usd ? (int)((cst + 1) / 2) : usd + (int)(cst - 2ll * usd));
         };
         const int d0 = first(cost * blockIdx.x / gridDim.x), d1 = first(cost * (blockIdx.x + 1) / gridDim.x);
-        for (int u = d0; u < d1 && !s.abort; ++u) issue(u, unit_of(u, usg, n, usd));
+        for (int u = d0; u < d1 && !s.abort; ++u) issue(u, unit_of<WF>(u, usg, n, usd));
         if (!s.abort) {
             const int slot = gi % kStages;
             if (mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1)) {
@@ -358,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 if (lane == 0) mbar_arrive(&s.rempty[rb]);
                 continue;
             }
-            const Unit un = unit_of(m >> 3, usg, n, usd);
+            const Unit un = unit_of<WF>(m >> 3, usg, n, usd);
             const float(*red)[2][128] = s.red[rb];
             if (un.kind == kGsh || un.kind == kGrt) {
                 const bool sh = un.kind == kGsh;
@@ -424,6 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     // ------------------------------ consumers ------------------------------
     const int g = lane >> 2, q = lane & 3;
     uint32_t B[16][4];
+    uint32_t Bm[2][4];          // Q2_K: sub-block sums per super-block (hi, lo)
     int bkind = -1, bseg = -2;  // what B holds
     bool dep = false;           // grid dependency resolved for this thread
     bool flushed = false;       // gate/up count of this CTA published
@@ -445,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             if ((!flushed && !marker(-2)) || !marker(-1)) fail(a, s);
             return;
         }
-        const Unit un = unit_of(u, usg, u < usg ? 0 : s.n_seg, usd);
+        const Unit un = unit_of<WF>(u, usg, u < usg ? 0 : s.n_seg, usd);
         if (un.kind != kGsh && !dep) {
             grid_dep_wait();
             dep = true;
@@ -460,7 +605,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 }
                 if (!wait_count(gu_done, (uint32_t)(usg + s.n_seg * kGuTiles), lane)) { fail(a, s); return; }
             }
-            if (un.kind == kGsh || un.kind == kGrt) {
+            if (Q2 && un.kind == kGrt) {  // x, this warp's 2 super-blocks of K
+                const int tok = min(g, a.T - 1);
+                q2k_load_b<2, false>(a.x + (int64_t)tok * kD + 512 * warp, a.xscale[tok].y, q, B, Bm);
+            } else if (Q2 && un.kind == kDrt) {  // h, this warp's super-block of K
+                const int e = s.seg_e[un.seg];
+                const int rbase = a.offsets[e], cnt = a.offsets[e + 1] - rbase;
+                const int row = rbase + min(g, cnt - 1);
+                const float sc = 1.0f / row_scale(__ldcg(&a.hmax[row]));
+                q2k_load_b<1, true>(a.h + (int64_t)row * kF + 256 * warp, sc, q, B, Bm);
+            } else if (un.kind == kGsh || un.kind == kGrt) {
                 const bool sh = un.kind == kGsh;
                 const int tok = min(g, a.T - 1);
                 const float inv = sh ? 1.f : a.xscale[tok].y;
@@ -509,6 +663,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 #pragma unroll
                         for (int m = 0; m < 2; ++m)
                             bf16_block(acc[m], st + 16384 * m, 16, 2 * warp + jj, g, q, B[2 * cc + jj]);
+        } else if (Q2 && un.kind == kGrt) {
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2)
+                    q2k_superblock(acc[m], st + 16384 * m, ss + 4096 * m, ss + kQDd + 1024 * m, 16, 64, 0,
+                                   2 * warp + s2, g, q, B + 8 * s2, Bm[s2]);
+        } else if (Q2 && un.kind == kDrt) {
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+                q2k_superblock(acc[t], st, ss, ss + kQDd, 32, 32, 16 * t, warp, g, q, B, Bm[0]);
         } else if (un.kind == kGrt) {
             uint32_t sw[2][2][2];
 #pragma unroll
@@ -762,7 +927,11 @@ cudaError_t set_smem_attrs() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (done[dev]) return cudaSuccess;
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(decode_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)))
+    if ((e = cudaFuncSetAttribute(decode_ffn_kernel<MOE_W_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kSmemBytes)))
+        return e;
+    if ((e = cudaFuncSetAttribute(decode_ffn_kernel<MOE_W_Q2K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kSmemBytes)))
         return e;
     if ((e = cudaFuncSetAttribute(decode_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLogitsSmem)))
         return e;
@@ -792,7 +961,8 @@ cudaError_t launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cuda
 
 bool decode_path_applies(const moe_dims &d) {
     // the tiling is written for d_model 4096, d_ff 2048 (and a shared d_ff of 2048)
-    return d.T >= 1 && d.T <= 8 && d.wfmt == MOE_W_MXFP4 && d.act == MOE_A_BF16 && d.d_model == kD &&
+    return d.T >= 1 && d.T <= 8 && (d.wfmt == MOE_W_MXFP4 || d.wfmt == MOE_W_Q2K) && d.act == MOE_A_BF16 &&
+           d.d_model == kD &&
            d.d_ff == kF && (d.d_ff_shared == 0 || d.d_ff_shared == 2048) && d.E <= kMaxE;
 }
 
@@ -828,18 +998,33 @@ cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uin
                               const WsLayout &L, cudaStream_t s, bool prepared) {
     cudaError_t e = set_smem_attrs();
     if (e != cudaSuccess) return e;
-    const Mxfp4Layout L1 = mxfp4_layout(d, MOE_MAT_W1), L2 = mxfp4_layout(d, MOE_MAT_W2);
     DecodeArgs a;
     memset(&a, 0, sizeof a);
     const uint8_t *p1 = static_cast<const uint8_t *>(w.w1), *p3 = static_cast<const uint8_t *>(w.w3),
                   *p2 = static_cast<const uint8_t *>(w.w2);
     const uint64_t r13 = (uint64_t)d.E * kF, r2 = (uint64_t)d.E * kD;
-    bool ok = make_chunked_map(&a.m1c, p1 + L1.codes, r13, kD / 2, 16, 8) &&
-              make_chunked_map(&a.m3c, p3 + L1.codes, r13, kD / 2, 16, 8) &&
-              make_chunked_map(&a.m2c, p2 + L2.codes, r2, kF / 2, 32, 8) &&
-              make_plain_map(&a.m1s, p1 + L1.srow, r13, kD / 32, 64, 16) &&
-              make_plain_map(&a.m3s, p3 + L1.srow, r13, kD / 32, 64, 16) &&
-              make_plain_map(&a.m2s, p2 + L2.srow, r2, kF / 32, 64, 32);
+    const bool q2 = d.wfmt == MOE_W_Q2K;
+    bool ok;
+    if (q2) {  // quants (64 B per 256 weights), sc|m bytes (16 B), (d, dmin) pairs (4 B)
+        const Q2kLayout L1 = q2k_layout(d, MOE_MAT_W1), L2 = q2k_layout(d, MOE_MAT_W2);
+        ok = make_chunked_map(&a.m1c, p1 + L1.qs, r13, kD / 4, 16, 8) &&
+             make_chunked_map(&a.m3c, p3 + L1.qs, r13, kD / 4, 16, 8) &&
+             make_chunked_map(&a.m2c, p2 + L2.qs, r2, kF / 4, 32, 4) &&
+             make_chunked_map(&a.m1s, p1 + L1.scm, r13, kD / 16, 16, 2) &&
+             make_chunked_map(&a.m3s, p3 + L1.scm, r13, kD / 16, 16, 2) &&
+             make_chunked_map(&a.m2s, p2 + L2.scm, r2, kF / 16, 32, 1) &&
+             make_plain_map(&a.m1d, p1 + L1.dd, r13, kD / 64, kD / 64, 16) &&
+             make_plain_map(&a.m3d, p3 + L1.dd, r13, kD / 64, kD / 64, 16) &&
+             make_plain_map(&a.m2d, p2 + L2.dd, r2, kF / 64, kF / 64, 32);
+    } else {
+        const Mxfp4Layout L1 = mxfp4_layout(d, MOE_MAT_W1), L2 = mxfp4_layout(d, MOE_MAT_W2);
+        ok = make_chunked_map(&a.m1c, p1 + L1.codes, r13, kD / 2, 16, 8) &&
+             make_chunked_map(&a.m3c, p3 + L1.codes, r13, kD / 2, 16, 8) &&
+             make_chunked_map(&a.m2c, p2 + L2.codes, r2, kF / 2, 32, 8) &&
+             make_plain_map(&a.m1s, p1 + L1.srow, r13, kD / 32, 64, 16) &&
+             make_plain_map(&a.m3s, p3 + L1.srow, r13, kD / 32, 64, 16) &&
+             make_plain_map(&a.m2s, p2 + L2.srow, r2, kF / 32, 64, 32);
+    }
     if (ok && shared_out)
         ok = make_chunked_map(&a.ms1, w.sw1, d.d_ff_shared, kD * 2, 16, 8) &&
              make_chunked_map(&a.ms3, w.sw3, d.d_ff_shared, kD * 2, 16, 8) &&
@@ -861,8 +1046,9 @@ cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uin
                                               a.counters);
         count_launches(1);
     }
-    if ((e = launch_pdl(decode_ffn_kernel, dim3(num_sms()), dim3(kThreads), kSmemBytes, s, a)) != cudaSuccess)
-        return e;
+    e = q2 ? launch_pdl(decode_ffn_kernel<MOE_W_Q2K>, dim3(num_sms()), dim3(kThreads), kSmemBytes, s, a)
+           : launch_pdl(decode_ffn_kernel<MOE_W_MXFP4>, dim3(num_sms()), dim3(kThreads), kSmemBytes, s, a);
+    if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
 }

@@ -37,12 +37,13 @@ __device__ __forceinline__ float block_dot(int wfmt, const uint8_t *packed, int6
         const uint32_t dd = reinterpret_cast<const uint32_t *>(packed + off_c)[sb];
         const float dv = __half2float(__ushort_as_half((uint16_t)(dd & 0xFFFF)));
         const float mv = __half2float(__ushort_as_half((uint16_t)(dd >> 16)));
-        const uint8_t *q = packed + off_a + sb * 64 + (kb % 8) * 8;
+        const uint32_t *qw = reinterpret_cast<const uint32_t *>(packed + off_a) + sb * 16;
         for (int h = 0; h < 2; ++h) {
             const uint8_t scm = packed[off_b + sb * 16 + (kb % 8) * 2 + h];
             const float ds = __fmul_rn(dv, (float)(scm & 15)), dm = __fmul_rn(mv, (float)(scm >> 4));
             for (int j = 0; j < 16; ++j) {
-                const int qq = (q[(16 * h + j) / 4] >> (2 * ((16 * h + j) % 4))) & 3;
+                const int e = (kb % 8) * 32 + 16 * h + j;  // quant index in the super-block
+                const int qq = (int)((qw[q2k_word(e)] >> q2k_bit(e)) & 3u);
                 acc = fmaf(a(kb * 32 + 16 * h + j), __fsub_rn(__fmul_rn(ds, (float)qq), dm), acc);
             }
         }

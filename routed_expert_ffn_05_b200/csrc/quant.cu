@@ -145,7 +145,13 @@ __global__ void pack_q2k_kernel(const uint8_t *__restrict__ in, int64_t nsb, uin
     if (sb >= nsb) return;
     const uint8_t *b = in + sb * 84;
     for (int i = 0; i < 16; ++i) scm[sb * 16 + i] = b[i];
-    for (int i = 0; i < 64; ++i) qs[sb * 64 + i] = b[16 + i];
+    uint32_t words[16] = {};
+    for (int e = 0; e < 256; ++e) {  // canonical: quant e at byte e / 4, bits 2 (e % 4)
+        const uint32_t q = (b[16 + e / 4] >> (2 * (e % 4))) & 3u;
+        words[q2k_word(e)] |= q << q2k_bit(e);
+    }
+    uint32_t *qw = reinterpret_cast<uint32_t *>(qs + sb * 64);
+    for (int i = 0; i < 16; ++i) qw[i] = words[i];
     dd[sb] = (uint32_t)b[80] | (uint32_t)b[81] << 8 | (uint32_t)b[82] << 16 | (uint32_t)b[83] << 24;
 }
 
@@ -184,7 +190,8 @@ __global__ void debug_dequant_kernel(const uint8_t *__restrict__ packed, int wfm
         const uint32_t dd = reinterpret_cast<const uint32_t *>(packed + off_c)[sb];
         const float dv = __half2float(__ushort_as_half((uint16_t)(dd & 0xFFFF)));
         const float mv = __half2float(__ushort_as_half((uint16_t)(dd >> 16)));
-        const int q = (packed[off_a + sb * 64 + j / 4] >> (2 * (j % 4))) & 3;
+        const uint32_t w = reinterpret_cast<const uint32_t *>(packed + off_a)[sb * 16 + q2k_word((int)j)];
+        const int q = (int)((w >> q2k_bit((int)j)) & 3u);
         const float a = __fmul_rn(__fmul_rn(dv, (float)(scm & 15)), (float)q);
         out[i] = __fsub_rn(a, __fmul_rn(mv, (float)(scm >> 4)));
     } else {
