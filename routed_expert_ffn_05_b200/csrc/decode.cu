@@ -43,7 +43,7 @@
 namespace moe {
 namespace {
 
-constexpr int kCW = 8;                    // consumer warps
+constexpr int kCW = 16;                   // consumer warps (each owns 1/16 of K)
 constexpr int kProducer = kCW;            // warp index of the producer
 constexpr int kEpilogue = kCW + 1;        // warp index of the epilogue warp
 constexpr int kThreads = (kCW + 2) * 32;
@@ -224,21 +224,25 @@ __device__ __forceinline__ uint32_t q2_pair(uint32_t w, uint32_t sc) {
 }
 __host__ __device__ constexpr float q2_pre(int k) { return k % 3 == 0 ? 1.0f : (k % 3 == 1 ? 0.25f : 0.0625f); }
 
-// One super-block (16 sub-blocks of 16) of 16 rows r0 + g, r0 + g + 8 of a
-// Q2_K box (quants: `rows` rows, 128-byte chunks; sc|m: same rows, chunked;
-// dd: row-major, `ddrow` bytes per row) against B (16 sub-blocks) and bm (the
-// sub-block sums as f16 hi + lo parts: bm[0..1] hi, bm[2..3] lo).
-// acc += d (sum_j sc_j q . x) - dmin (sum_j m_j xsum_j).
+// One super-block (16 sub-blocks of 16), or half of one (HALF 0: sub-blocks
+// 0..7, HALF 1: 8..15; HALF -1: all), of 16 rows r0 + g, r0 + g + 8 of a Q2_K
+// box (quants: `rows` rows, 128-byte chunks; sc|m: same rows, chunked; dd:
+// row-major, `ddrow` bytes per row) against B (this part's sub-blocks) and bm
+// (sub-block sums as f16 hi + lo parts: bm[0..1] hi, bm[2..3] lo).
+// acc += d (sum_j sc_j q . x) - dmin (sum_j m_j xsum_j) over the part.
+template <int HALF>
 __device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, const uint8_t *scm,
                                                const uint8_t *dd, int rows, int ddrow, int r0, int sb, int g,
                                                int q, const uint32_t (*B)[4], const uint32_t bm[4]) {
+    constexpr int G0 = HALF == 1 ? 2 : 0, NG = HALF < 0 ? 4 : 2;
     const int rg = r0 + g, rh = r0 + g + 8;
     const uint4 ml = lds128(scm + swz_off((sb * 16) / 128, rows, rg, sb % 8));
     const uint4 mh = lds128(scm + swz_off((sb * 16) / 128, rows, rh, sb % 8));
     const uint32_t sl[4] = {ml.x, ml.y, ml.z, ml.w}, sh[4] = {mh.x, mh.y, mh.z, mh.w};
     float tm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int G = 0; G < 4; ++G) {
+    for (int Gi = 0; Gi < NG; ++Gi) {
+        const int G = G0 + Gi;
         const int c = (sb * 64) / 128, u = 4 * (sb & 1) + G;
         const uint32_t wl = lds32(qs + swz_off(c, rows, rg, u) + 4 * q);
         const uint32_t wh = lds32(qs + swz_off(c, rows, rh, u) + 4 * q);
@@ -252,19 +256,21 @@ __device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, 
                 case 2: a0 = q2_pair<4>(wl, cl); a1 = q2_pair<4>(wh, ch); a2 = q2_pair<5>(wl, cl); a3 = q2_pair<5>(wh, ch); break;
                 default: a0 = q2_pair<6>(wl, cl); a1 = q2_pair<6>(wh, ch); a2 = q2_pair<7>(wl, cl); a3 = q2_pair<7>(wh, ch);
             }
-            const int j = 4 * G + jj;
-            mma_f16_16816(tm, a0, a1, a2, a3, B[j >> 1][2 * (j & 1)], B[j >> 1][2 * (j & 1) + 1]);
+            const int jl = 4 * Gi + jj;  // sub-block within this part
+            mma_f16_16816(tm, a0, a1, a2, a3, B[jl >> 1][2 * (jl & 1)], B[jl >> 1][2 * (jl & 1) + 1]);
         }
     }
-    // minimum term: A = m of sub-blocks 2q, 2q+1 (k-slots 2q, 2q+1) and 2q+8, 2q+9
+    // minimum term: A = m of sub-blocks 2q, 2q+1 (k-slots 2q, 2q+1) and 2q+8, 2q+9;
+    // a half keeps only its own sub-blocks
     auto mpair = [&](uint32_t w) {  // bytes 0, 1 of w -> their high nibbles as an f16 subnormal pair
         return ((w >> 4) & 0xFu) | ((w << 4) & 0xF0000u);
     };
     const int sh16 = 16 * (q & 1);
     const uint32_t lA = (q < 2 ? ml.x : ml.y) >> sh16, lB = (q < 2 ? ml.z : ml.w) >> sh16;
     const uint32_t hA = (q < 2 ? mh.x : mh.y) >> sh16, hB = (q < 2 ? mh.z : mh.w) >> sh16;
+    const uint32_t ma0 = HALF == 1 ? 0u : mpair(lA), ma1 = HALF == 1 ? 0u : mpair(hA);
+    const uint32_t ma2 = HALF == 0 ? 0u : mpair(lB), ma3 = HALF == 0 ? 0u : mpair(hB);
     float tn[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t ma0 = mpair(lA), ma1 = mpair(hA), ma2 = mpair(lB), ma3 = mpair(hB);
     mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[0], bm[1]);
     mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[2], bm[3]);
     const uint32_t dl = lds32(dd + rg * ddrow + 4 * sb), dh = lds32(dd + rh * ddrow + 4 * sb);
@@ -279,47 +285,45 @@ __device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, 
     acc[3] = fmaf(-m1, tn[3], fmaf(d1, tm[3], acc[3]));
 }
 
-// B fragments of `nsb` super-blocks (16 sub-blocks each) of one activation row
-// (bf16, scaled by `inv`): k-slot pre-scale 4^-(k % 3), the elements of lane q
-// as described above; bm gets the sub-block sums (scaled by 2^-5) of
-// sub-blocks 2q, 2q+1, 2q+8, 2q+9 of each super-block, each split into an f16
-// part and the f16 of its remainder (together ~22 bits: the minimum term
-// nearly cancels the main term, so its sums need more than f16).
-template <int NSB, bool CG>
-__device__ __forceinline__ void q2k_load_b(const uint16_t *row, float inv, int q, uint32_t (*B)[4],
-                                           uint32_t (*bm)[4]) {
+// B fragments of one super-block, or half of one (HALF as above), of an
+// activation row (bf16 at `row` = the super-block's first element, scaled by
+// `inv`): k-slot pre-scale 4^-(k % 3), the elements of lane q as described
+// above; bm gets the sums (scaled by 2^-5) of sub-blocks 2q, 2q+1, 2q+8, 2q+9
+// that lie in the part (zero otherwise), each split into an f16 part and the
+// f16 of its remainder (together ~22 bits: the minimum term nearly cancels
+// the main term, so its sums need more than f16).
+template <int HALF, bool CG>
+__device__ __forceinline__ void q2k_load_b(const uint16_t *row, float inv, int q, uint32_t (*B)[4], uint32_t bm[4]) {
+    constexpr int J0 = HALF == 1 ? 8 : 0, NJ = HALF < 0 ? 16 : 8;
+    float keep[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int s2 = 0; s2 < NSB; ++s2) {
-        float keep[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const uint16_t *src = row + 256 * s2 + 16 * j + 4 * q;
-            const uint2 v = CG ? __ldcg(reinterpret_cast<const uint2 *>(src)) : __ldg(reinterpret_cast<const uint2 *>(src));
-            const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xFFFF0000u);
-            const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xFFFF0000u);
-            const int jl = 16 * s2 + j;
-            const float c0 = inv * q2_pre(2 * (j & 3)), c1 = inv * q2_pre(2 * (j & 3) + 1);
-            B[jl >> 1][2 * (jl & 1)] = f32x2_to_f16x2(x0 * c0, x1 * c0);
-            B[jl >> 1][2 * (jl & 1) + 1] = f32x2_to_f16x2(x2 * c1, x3 * c1);
-            float ps = (x0 + x1) + (x2 + x3);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-            if (j < 8 && (j >> 1) == q) keep[j & 1] = ps;
-            if (j >= 8 && ((j - 8) >> 1) == q) keep[2 + (j & 1)] = ps;
-        }
-        const float xs = inv * 0.03125f;
-        float hi[4], lo[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float v = keep[i] * xs;
-            hi[i] = __half2float(__float2half_rn(v));
-            lo[i] = v - hi[i];
-        }
-        bm[s2][0] = f32x2_to_f16x2(hi[0], hi[1]);
-        bm[s2][1] = f32x2_to_f16x2(hi[2], hi[3]);
-        bm[s2][2] = f32x2_to_f16x2(lo[0], lo[1]);
-        bm[s2][3] = f32x2_to_f16x2(lo[2], lo[3]);
+    for (int ji = 0; ji < NJ; ++ji) {
+        const int j = J0 + ji;
+        const uint16_t *src = row + 16 * j + 4 * q;
+        const uint2 v = CG ? __ldcg(reinterpret_cast<const uint2 *>(src)) : __ldg(reinterpret_cast<const uint2 *>(src));
+        const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xFFFF0000u);
+        const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xFFFF0000u);
+        const float c0 = inv * q2_pre(2 * (j & 3)), c1 = inv * q2_pre(2 * (j & 3) + 1);
+        B[ji >> 1][2 * (ji & 1)] = f32x2_to_f16x2(x0 * c0, x1 * c0);
+        B[ji >> 1][2 * (ji & 1) + 1] = f32x2_to_f16x2(x2 * c1, x3 * c1);
+        float ps = (x0 + x1) + (x2 + x3);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+        if (j < 8 && (j >> 1) == q) keep[j & 1] = ps;
+        if (j >= 8 && ((j - 8) >> 1) == q) keep[2 + (j & 1)] = ps;
     }
+    const float xs = inv * 0.03125f;
+    float hi[4], lo[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float v = keep[i] * xs;
+        hi[i] = __half2float(__float2half_rn(v));
+        lo[i] = v - hi[i];
+    }
+    bm[0] = f32x2_to_f16x2(hi[0], hi[1]);
+    bm[1] = f32x2_to_f16x2(hi[2], hi[3]);
+    bm[2] = f32x2_to_f16x2(lo[0], lo[1]);
+    bm[3] = f32x2_to_f16x2(lo[2], lo[3]);
 }
 
 template <int WF>
@@ -566,9 +570,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     }
 
     // ------------------------------ consumers ------------------------------
+    // Warp w owns 1/16 of K in every unit: shared gate/up 1 block of 32 per
+    // stage (8 stages of K 512), routed MXFP4 gate/up 4 blocks per stage (2 of
+    // K 2048), shared down 2 blocks per stage (2 of K 1024), routed MXFP4
+    // down 4 blocks (K 2048), Q2_K gate/up one super-block, Q2_K down half of
+    // one. B holds this warp's activation fragments for the unit's kind.
     const int g = lane >> 2, q = lane & 3;
-    uint32_t B[16][4];
-    uint32_t Bm[2][4];          // Q2_K: sub-block sums per super-block (hi, lo)
+    uint32_t B[8][4];
+    uint32_t Bm[4];             // Q2_K: sub-block sums (hi, lo)
     int bkind = -1, bseg = -2;  // what B holds
     bool dep = false;           // grid dependency resolved for this thread
     bool flushed = false;       // gate/up count of this CTA published
@@ -595,9 +604,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             grid_dep_wait();
             dep = true;
         }
-        if (un.kind != bkind || un.seg != bseg) {
+        // B depends on the kind, and for down units on the expert (its h rows)
+        const int useg = (un.kind == kDrt) ? un.seg : -1;
+        if (un.kind != bkind || useg != bseg) {
             bkind = un.kind;
-            bseg = un.seg;
+            bseg = useg;
             if (un.kind == kDsh || un.kind == kDrt) {  // every gate/up unit must be complete
                 if (!flushed) {
                     if (!marker(-2)) { fail(a, s); return; }
@@ -605,24 +616,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 }
                 if (!wait_count(gu_done, (uint32_t)(usg + s.n_seg * kGuTiles), lane)) { fail(a, s); return; }
             }
-            if (Q2 && un.kind == kGrt) {  // x, this warp's 2 super-blocks of K
+            if (Q2 && un.kind == kGrt) {  // x: super-block `warp` of K
                 const int tok = min(g, a.T - 1);
-                q2k_load_b<2, false>(a.x + (int64_t)tok * kD + 512 * warp, a.xscale[tok].y, q, B, Bm);
-            } else if (Q2 && un.kind == kDrt) {  // h, this warp's super-block of K
+                q2k_load_b<-1, false>(a.x + (int64_t)tok * kD + 256 * warp, a.xscale[tok].y, q, B, Bm);
+            } else if (Q2 && un.kind == kDrt) {  // h: half (warp & 1) of super-block warp / 2
                 const int e = s.seg_e[un.seg];
                 const int rbase = a.offsets[e], cnt = a.offsets[e + 1] - rbase;
                 const int row = rbase + min(g, cnt - 1);
                 const float sc = 1.0f / row_scale(__ldcg(&a.hmax[row]));
-                q2k_load_b<1, true>(a.h + (int64_t)row * kF + 256 * warp, sc, q, B, Bm);
+                const uint16_t *hr = a.h + (int64_t)row * kF + 256 * (warp >> 1);
+                if (warp & 1) q2k_load_b<1, true>(hr, sc, q, B, Bm);
+                else q2k_load_b<0, true>(hr, sc, q, B, Bm);
             } else if (un.kind == kGsh || un.kind == kGrt) {
                 const bool sh = un.kind == kGsh;
                 const int tok = min(g, a.T - 1);
                 const float inv = sh ? 1.f : a.xscale[tok].y;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    // shared: stage j/2 holds blocks 16(j/2)..+15 of K; this warp takes 2w, 2w+1
-                    // routed: stage j/8 holds blocks 64(j/8)..+63; this warp takes 8w..8w+7
-                    const int kb = sh ? 16 * (j / 2) + 2 * warp + (j & 1) : 64 * (j / 8) + 8 * warp + (j & 7);
+                for (int j = 0; j < 8; ++j) {
+                    // shared: stage j holds blocks 16 j .. +15 of K; this warp takes 16 j + w
+                    // routed: stage j/4 holds blocks 64 (j/4) .. +63; this warp takes 4w .. 4w+3
+                    const int kb = sh ? 16 * j + warp : 64 * (j / 4) + 4 * warp + (j & 3);
                     const uint4 v = ldg128(a.x + (int64_t)tok * kD + 32 * kb + 8 * q);
                     const uint32_t raw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -631,8 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             } else if (un.kind == kDsh) {
                 const int tok = min(g, a.T - 1);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {  // stage j/4 holds blocks 32(j/4)..+31; this warp 4w..4w+3
-                    const uint4 v = ldcg128(a.hs + (int64_t)tok * a.Fs + 32 * (32 * (j / 4) + 4 * warp + (j & 3)) + 8 * q);
+                for (int j = 0; j < 4; ++j) {  // stage j/2 holds blocks 32 (j/2) .. +31; this warp 2w, 2w+1
+                    const uint4 v = ldcg128(a.hs + (int64_t)tok * a.Fs + 32 * (32 * (j / 2) + 2 * warp + (j & 1)) + 8 * q);
                     B[j][0] = v.x; B[j][1] = v.y; B[j][2] = v.z; B[j][3] = v.w;
                 }
             } else {
@@ -641,8 +654,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 const int row = rbase + min(g, cnt - 1);
                 const float sc = 1.0f / row_scale(__ldcg(&a.hmax[row]));
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 v = ldcg128(a.h + (int64_t)row * kF + 32 * (8 * warp + j) + 8 * q);
+                for (int j = 0; j < 4; ++j) {  // blocks 4w .. 4w+3 of K
+                    const uint4 v = ldcg128(a.h + (int64_t)row * kF + 32 * (4 * warp + j) + 8 * q);
                     B[j][0] = bf16x2_to_f16x2(v.x, sc);
                     B[j][1] = bf16x2_to_f16x2(v.y, sc);
                     B[j][2] = bf16x2_to_f16x2(v.z, sc);
@@ -659,57 +672,51 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             for (int cc = 0; cc < 8; ++cc)
                 if (cc == c)
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-                        for (int m = 0; m < 2; ++m)
-                            bf16_block(acc[m], st + 16384 * m, 16, 2 * warp + jj, g, q, B[2 * cc + jj]);
+                    for (int m = 0; m < 2; ++m) bf16_block(acc[m], st + 16384 * m, 16, warp, g, q, B[cc]);
         } else if (Q2 && un.kind == kGrt) {
 #pragma unroll
             for (int m = 0; m < 2; ++m)
-#pragma unroll
-                for (int s2 = 0; s2 < 2; ++s2)
-                    q2k_superblock(acc[m], st + 16384 * m, ss + 4096 * m, ss + kQDd + 1024 * m, 16, 64, 0,
-                                   2 * warp + s2, g, q, B + 8 * s2, Bm[s2]);
+                q2k_superblock<-1>(acc[m], st + 16384 * m, ss + 4096 * m, ss + kQDd + 1024 * m, 16, 64, 0, warp, g,
+                                   q, B, Bm);
         } else if (Q2 && un.kind == kDrt) {
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
-                q2k_superblock(acc[t], st, ss, ss + kQDd, 32, 32, 16 * t, warp, g, q, B, Bm[0]);
+            for (int t = 0; t < 2; ++t) {
+                if (warp & 1) q2k_superblock<1>(acc[t], st, ss, ss + kQDd, 32, 32, 16 * t, warp >> 1, g, q, B, Bm);
+                else q2k_superblock<0>(acc[t], st, ss, ss + kQDd, 32, 32, 16 * t, warp >> 1, g, q, B, Bm);
+            }
         } else if (un.kind == kGrt) {
-            uint32_t sw[2][2][2];
+            // this warp's 4 blocks: 16-byte units 4 (w & 1) .. +3 of chunk w / 2; scale word w of each row
+            uint32_t sw[2][2];
 #pragma unroll
             for (int m = 0; m < 2; ++m)
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) sw[m][hh][i] = lds32(ss + 1024 * m + (g + 8 * hh) * 64 + 4 * (2 * warp + i));
+                for (int hh = 0; hh < 2; ++hh) sw[m][hh] = lds32(ss + 1024 * m + (g + 8 * hh) * 64 + 4 * warp);
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc)
                 if (cc == c)
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj)
+                    for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
                         for (int m = 0; m < 2; ++m)
-                            mxfp4_block(acc[m], st + 16384 * m, 16, warp, jj, 0, g, q, sw[m][0][jj / 4],
-                                        sw[m][1][jj / 4], jj % 4, B[8 * cc + jj]);
+                            mxfp4_block(acc[m], st + 16384 * m, 16, warp >> 1, 4 * (warp & 1) + jj, 0, g, q, sw[m][0],
+                                        sw[m][1], jj, B[4 * cc + jj]);
         } else if (un.kind == kDsh) {
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc)
                 if (cc == c)
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) bf16_block(acc[0], st, 16, 4 * warp + jj, g, q, B[4 * cc + jj]);
+                    for (int jj = 0; jj < 2; ++jj) bf16_block(acc[0], st, 16, 2 * warp + jj, g, q, B[2 * cc + jj]);
         } else {
-            uint32_t sw[2][2][2];
+            uint32_t sw[2][2];
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
+                for (int hh = 0; hh < 2; ++hh) sw[t][hh] = lds32(ss + (16 * t + g + 8 * hh) * 64 + 4 * warp);
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) sw[t][hh][i] = lds32(ss + (16 * t + g + 8 * hh) * 64 + 4 * (2 * warp + i));
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
+            for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
                 for (int t = 0; t < 2; ++t)
-                    mxfp4_block(acc[t], st, 32, warp, jj, 16 * t, g, q, sw[t][0][jj / 4], sw[t][1][jj / 4], jj % 4,
+                    mxfp4_block(acc[t], st, 32, warp >> 1, 4 * (warp & 1) + jj, 16 * t, g, q, sw[t][0], sw[t][1], jj,
                                 B[jj]);
         }
         __syncwarp();
