@@ -77,7 +77,7 @@ struct DecodeArgs {
     uint16_t *hs;            // shared hidden [T][Fs] bf16
     float *out_rows;         // [S][d]
     float *shared_out;       // [T][d]
-    uint32_t *counters;      // [0] work queue, [1] shared gate/up tiles done, [2+e] expert e tiles done
+    uint32_t *counters;      // [0] work queue, [1] shared gate/up tiles done, [2+s] gate/up tiles done of active expert s
     int *err;
 };
 
@@ -202,6 +202,12 @@ __device__ __forceinline__ void put_partial(float *r, int rg, int q, const float
 // bf16 pair -> f16 pair scaled by an exact power of two.
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, float sc) {
     return f32x2_to_f16x2(__uint_as_float(v << 16) * sc, __uint_as_float(v & 0xFFFF0000u) * sc);
+}
+
+__device__ __forceinline__ uint32_t warp_max_bits(uint32_t v) {
+    uint32_t r;
+    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+    return r;
 }
 
 __device__ __forceinline__ float row_scale(uint32_t hm) {  // 2^p with max |h| * 2^-p in [2^14, 2^15)
@@ -348,9 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     grid_dep_launch();
     const int usg = a.Fs > 0 ? a.Fs / 16 : 0;  // shared gate/up units (no routing needed)
     const int usd = a.Fs > 0 ? kDshTiles : 0;
-    // finished gate/up units, published once per CTA (flush marker below);
-    // down units wait for all of them
-    uint32_t *gu_done = a.counters + 1;
+    // finished gate/up tiles, published per expert (and for the shared expert)
+    // by the epilogue; a down unit waits only for its own expert's tiles
+    uint32_t *sh_done = a.counters + 1, *seg_done = a.counters + 2;
 
     // ------------------------------ producer ------------------------------
     if (warp == kProducer) {
@@ -490,7 +496,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             for (int i = 0; i < s.ep_cnt[sg]; ++i) s.ep_tok[sg][i] = (uint8_t)(a.perm[s.ep_rbase[sg] + i] / a.k);
         if (lane < a.T) s.ep_xs[lane] = a.xscale[lane].x;
         __syncwarp();
-        uint32_t finished = 0;  // gate/up units finished here and not yet published
+        // gate/up tiles finished here and not yet published: shared, and routed of segment pseg
+        uint32_t sh_fin = 0, r_fin = 0;
+        int pseg = -1;
+        auto publish = [&]() {  // this warp's h / hs writes, then the counts
+            if (!sh_fin && !r_fin) return;
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) {
+                if (sh_fin) atomicAdd(sh_done, sh_fin);
+                if (r_fin) atomicAdd(seg_done + pseg, r_fin);
+            }
+            sh_fin = r_fin = 0;
+        };
         int dseg = -1;
         float dsc = 1.f;        // lane i < 8: output scale of row i of segment dseg
         for (int ru = 0;; ++ru) {
@@ -498,70 +516,84 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             if (!mbar_wait(&s.rfull[rb], (ru >> 1) & 1)) { fail(a, s); return; }
             const int m = s.rmeta[rb];
             if (m == -1) return;
-            if (m == -2) {  // publish: this CTA's h / hs writes, then its count
-                __threadfence();
-                __syncwarp();
-                if (lane == 0 && finished) atomicAdd(gu_done, finished);
-                finished = 0;
+            if (m == -2) {  // before this CTA's first down unit: publish everything
+                publish();
                 if (lane == 0) mbar_arrive(&s.rempty[rb]);
                 continue;
             }
             const Unit un = unit_of<WF>(m >> 3, usg, n, usd);
             const float(*red)[2][128] = s.red[rb];
+            // Partial tiles are [row][column] per consumer warp; each lane sums
+            // 4 columns of one row across the warps with 16-byte loads.
+            auto sum4 = [&](int mat, int off) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int w = 0; w < kCW; ++w) {
+                    const float4 p = *reinterpret_cast<const float4 *>(&red[w][mat][off]);
+                    v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+                }
+                return v;
+            };
+            auto pick = [](const float4 &v, int c) { return c == 0 ? v.x : (c == 1 ? v.y : (c == 2 ? v.z : v.w)); };
             if (un.kind == kGsh || un.kind == kGrt) {
-                const bool sh = un.kind == kGsh;
-                const int rbase = sh ? 0 : s.ep_rbase[un.seg], cnt = sh ? a.T : s.ep_cnt[un.seg];
-                for (int o = lane; o < 16 * 8; o += 32) {
-                    const int row = o & 15, i = o >> 4;  // i: token (shared) or row of the expert (routed)
-                    uint32_t hb = 0;
-                    if (i < cnt) {
-                        const int tok = sh ? i : s.ep_tok[un.seg][i];
-                        float gs = 0.f, us = 0.f;
+                // lane: row l / 2 of the 16-row tile, columns 4 (l % 2) .. +3
+                const int row = lane >> 1, half = lane & 1, col = 16 * un.tile + row;
+                const float4 g4 = sum4(0, row * 8 + 4 * half), u4 = sum4(1, row * 8 + 4 * half);
+                if (un.kind == kGsh) {
 #pragma unroll
-                        for (int w = 0; w < kCW; ++w) {
-                            gs += red[w][0][row * 8 + tok];
-                            us += red[w][1][row * 8 + tok];
-                        }
-                        if (!sh) {
-                            gs *= s.ep_xs[tok];
-                            us *= s.ep_xs[tok];
-                        }
-                        hb = f32_to_bf16_rne(silu_f32(gs) * us);
-                        const int col = 16 * un.tile + row;
-                        if (sh) a.hs[(int64_t)tok * a.Fs + col] = (uint16_t)hb;
-                        else a.h[(int64_t)(rbase + i) * kF + col] = (uint16_t)hb;
+                    for (int c = 0; c < 4; ++c) {
+                        const int tok = 4 * half + c;
+                        if (tok < a.T)
+                            a.hs[(int64_t)tok * a.Fs + col] =
+                                f32_to_bf16_rne(silu_f32(pick(g4, c)) * pick(u4, c));
                     }
-                    if (!sh) {  // one atomic per (row of the expert) per half-warp
-                        uint32_t mx = (hb & 0x7FFFu) << 16;
-#pragma unroll
-                        for (int off = 8; off > 0; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                        if ((lane & 15) == 0 && i < cnt) atomicMax(&a.hmax[rbase + i], mx);
+                } else {
+                    const int rbase = s.ep_rbase[un.seg], cnt = s.ep_cnt[un.seg];
+                    for (int i = 0; i < cnt; ++i) {  // the expert's rows; column = the row's token
+                        const int tok = s.ep_tok[un.seg][i];
+                        const bool mine = (tok >> 2) == half;
+                        uint32_t hb = 0;
+                        if (mine) {
+                            const float xs = s.ep_xs[tok];
+                            hb = f32_to_bf16_rne(silu_f32(pick(g4, tok & 3) * xs) * (pick(u4, tok & 3) * xs));
+                            a.h[(int64_t)(rbase + i) * kF + col] = (uint16_t)hb;
+                        }
+                        const uint32_t mx = warp_max_bits((hb & 0x7FFFu) << 16);
+                        if (lane == 0) atomicMax(&a.hmax[rbase + i], mx);
                     }
                 }
-                ++finished;
+                if (un.kind == kGsh) {
+                    ++sh_fin;
+                } else {
+                    if (un.seg != pseg) {  // a new expert: the previous one's count goes out
+                        publish();
+                        pseg = un.seg;
+                    }
+                    ++r_fin;
+                }
             } else if (un.kind == kDsh) {
-                for (int o = lane; o < 16 * a.T; o += 32) {
-                    const int row = o & 15, tok = o >> 4;
-                    float v = 0.f;
+                const int row = lane >> 1, half = lane & 1;
+                const float4 v4 = sum4(0, row * 8 + 4 * half);
 #pragma unroll
-                    for (int w = 0; w < kCW; ++w) v += red[w][0][row * 8 + tok];
-                    a.shared_out[(int64_t)tok * kD + 16 * un.tile + row] = v;
+                for (int c = 0; c < 4; ++c) {
+                    const int tok = 4 * half + c;
+                    if (tok < a.T) a.shared_out[(int64_t)tok * kD + 16 * un.tile + row] = pick(v4, c);
                 }
             } else {
+                // lane = row of the 32-row tile; columns = the expert's rows
                 const int rbase = s.ep_rbase[un.seg], cnt = s.ep_cnt[un.seg];
                 if (un.seg != dseg) {
                     dseg = un.seg;
                     dsc = lane < cnt ? row_scale(__ldcg(&a.hmax[rbase + lane])) : 1.f;
                 }
-                for (int o = lane; o < 32 * 8; o += 32) {
-                    const int row = o & 31, i = o >> 5;
-                    const float sc = __shfl_sync(0xffffffffu, dsc, i);
-                    if (i < cnt) {
-                        float v = 0.f;
+                const int t = lane >> 4, r16 = lane & 15;
+                const float4 lo = sum4(t, r16 * 8), hi = sum4(t, r16 * 8 + 4);
 #pragma unroll
-                        for (int w = 0; w < kCW; ++w) v += red[w][row >> 4][(row & 15) * 8 + i];
-                        a.out_rows[(int64_t)(rbase + i) * kD + 32 * un.tile + row] = v * sc;
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    const float sc = __shfl_sync(0xffffffffu, dsc, i);
+                    if (i < cnt)
+                        a.out_rows[(int64_t)(rbase + i) * kD + 32 * un.tile + lane] =
+                            (i < 4 ? pick(lo, i) : pick(hi, i - 4)) * sc;
                 }
             }
             __syncwarp();
@@ -614,7 +646,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     if (!marker(-2)) { fail(a, s); return; }
                     flushed = true;
                 }
-                if (!wait_count(gu_done, (uint32_t)(usg + s.n_seg * kGuTiles), lane)) { fail(a, s); return; }
+                const bool ok = un.kind == kDsh ? wait_count(sh_done, (uint32_t)usg, lane)
+                                                : wait_count(seg_done + un.seg, (uint32_t)kGuTiles, lane);
+                if (!ok) { fail(a, s); return; }
             }
             if (Q2 && un.kind == kGrt) {  // x: super-block `warp` of K
                 const int tok = min(g, a.T - 1);
