@@ -154,8 +154,8 @@ def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=
     xs, toks = [], []
     for b in range(batches):
         c = cfg.with_T(T)
-        xs.append(torch.from_numpy(synth.make_x(c, 0, 1000 * rank + b).astype(np.int16)).to(dev))
-        toks.append(torch.from_numpy(synth.make_token_ids(c, 0, 1000 * rank + b)).to(dev)
+        xs.append(torch.from_numpy(synth.make_x(c, 0, batch_index(rank, b)).astype(np.int16)).to(dev))
+        toks.append(torch.from_numpy(synth.make_token_ids(c, 0, batch_index(rank, b))).to(dev)
                     if cfg.route == "hash" else None)
     y = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -219,11 +219,23 @@ def barrier(torch, world):
 
 
 def max_over_ranks(torch, world, v):
+    """The slowest rank's value (every rank gets it); NCCL on GPUs, gloo on CPU."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def batch_index(rank, b):
+    """Seeded batch id of rank `rank`'s b-th rotating batch: replicas never share inputs."""
+    return 1000 * rank + b
+
+
+def job_value(world, tokens_per_step, steps, max_seconds):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_step * steps / max_seconds
 
 
 class Clocks:
@@ -388,7 +400,7 @@ def main():
     r = measure(M, torch, layer, T, args.steps, args.warmup, rank, world)
     ck = clocks.stop()
     total_s = max_over_ranks(torch, world, sum(r["ms"]) / 1000.0)
-    value = world * T * args.steps / total_s
+    value = job_value(world, T, args.steps, total_s)
     ms_per_step = 1000.0 * total_s / args.steps
 
     if not args.no_e2e:
@@ -430,7 +442,7 @@ def main():
                    "l2": "flushed between steps (256 MB write), flush outside the timed events",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof,
-        "e2e": {"value": world * T * args.steps / e2e_s, "unit": UNIT,
+        "e2e": {"value": job_value(world, T, args.steps, e2e_s), "unit": UNIT,
                 "h2d_bytes_per_step": T * cfg.d * 2 + (T * 4 if cfg.route == "hash" else 0),
                 "d2h_bytes_per_step": T * cfg.d * 4},
         "gpu_launches": r["launches"], "gpu_launches_per_step": r["launches"] / args.steps,
