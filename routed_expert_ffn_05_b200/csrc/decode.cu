@@ -169,8 +169,8 @@ __device__ __forceinline__ void mxfp4_block(float acc[4], const uint8_t *box, in
     uint32_t al[4], ah[4];
     e2m1x8_to_f16x8(lds32(box + swz_off(chunk, rows, r0 + g, unit) + 4 * q), al);
     e2m1x8_to_f16x8(lds32(box + swz_off(chunk, rows, r0 + g + 8, unit) + 4 * q), ah);
-    float t[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_f16_16816(t, al[0], ah[0], al[1], ah[1], b[0], b[1]);
+    float t[4];
+    mma_f16_16816_z(t, al[0], ah[0], al[1], ah[1], b[0], b[1]);
     mma_f16_16816(t, al[2], ah[2], al[3], ah[3], b[2], b[3]);
     const float sl = e8m0_fast(sw_lo, sj), sh = e8m0_fast(sw_hi, sj);
     acc[0] = fmaf(sl, t[0], acc[0]);
@@ -245,7 +245,7 @@ __device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, 
     const uint4 ml = lds128(scm + swz_off((sb * 16) / 128, rows, rg, sb % 8));
     const uint4 mh = lds128(scm + swz_off((sb * 16) / 128, rows, rh, sb % 8));
     const uint32_t sl[4] = {ml.x, ml.y, ml.z, ml.w}, sh[4] = {mh.x, mh.y, mh.z, mh.w};
-    float tm[4] = {0.f, 0.f, 0.f, 0.f};
+    float tm[4];
 #pragma unroll
     for (int Gi = 0; Gi < NG; ++Gi) {
         const int G = G0 + Gi;
@@ -263,7 +263,8 @@ __device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, 
                 default: a0 = q2_pair<6>(wl, cl); a1 = q2_pair<6>(wh, ch); a2 = q2_pair<7>(wl, cl); a3 = q2_pair<7>(wh, ch);
             }
             const int jl = 4 * Gi + jj;  // sub-block within this part
-            mma_f16_16816(tm, a0, a1, a2, a3, B[jl >> 1][2 * (jl & 1)], B[jl >> 1][2 * (jl & 1) + 1]);
+            if (jl == 0) mma_f16_16816_z(tm, a0, a1, a2, a3, B[0][0], B[0][1]);
+            else mma_f16_16816(tm, a0, a1, a2, a3, B[jl >> 1][2 * (jl & 1)], B[jl >> 1][2 * (jl & 1) + 1]);
         }
     }
     // minimum term: A = m of sub-blocks 2q, 2q+1 (k-slots 2q, 2q+1) and 2q+8, 2q+9;
@@ -276,8 +277,8 @@ __device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, 
     const uint32_t hA = (q < 2 ? mh.x : mh.y) >> sh16, hB = (q < 2 ? mh.z : mh.w) >> sh16;
     const uint32_t ma0 = HALF == 1 ? 0u : mpair(lA), ma1 = HALF == 1 ? 0u : mpair(hA);
     const uint32_t ma2 = HALF == 0 ? 0u : mpair(lB), ma3 = HALF == 0 ? 0u : mpair(hB);
-    float tn[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[0], bm[1]);
+    float tn[4];
+    mma_f16_16816_z(tn, ma0, ma1, ma2, ma3, bm[0], bm[1]);
     mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[2], bm[3]);
     const uint32_t dl = lds32(dd + rg * ddrow + 4 * sb), dh = lds32(dd + rh * ddrow + 4 * sb);
     // 2^24 undoes the subnormal encoding; 2^5 the sub-block-sum pre-scale

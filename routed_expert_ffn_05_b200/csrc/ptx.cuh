@@ -161,11 +161,23 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
     return r;
 }
 
-// Byte j of a word of E8M0 scales -> fp32 2^(e-127) as a bit pattern. Exact
-// for bytes 1..254; byte 0 gives 0 and 0xFF gives +Inf (neither is produced by
-// the quantiser; the exact decode lives in the dequantiser).
+// Byte j of a word of E8M0 scales -> fp32 2^(e-127) as a bit pattern (one
+// shift and one mask: the byte lands on the exponent field). Exact for bytes
+// 1..254; byte 0 gives 0 and 0xFF gives +Inf (neither is produced by the
+// quantiser; the exact decode lives in the dequantiser).
 __device__ __forceinline__ float e8m0_fast(uint32_t word, int j) {
-    return __uint_as_float(((word >> (8 * j)) & 0xFFu) << 23);
+    const uint32_t v = j < 3 ? word << (23 - 8 * j) : word >> 1;
+    return __uint_as_float(v & 0x7F800000u);
+}
+
+// D = A(16x16, row) * B(16x8, col) with a zero accumulator input.
+__device__ __forceinline__ void mma_f16_16816_z(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 }  // namespace moe
