@@ -17,7 +17,9 @@
 //    tile) into two 128-column fp32 accumulators, so SwiGLU pairs g and u in
 //    the same thread after tcgen05.ld; the h block amax along F (across the
 //    warp's 32 lanes = 32 consecutive weight rows) is one redux.sync;
-//  - down: one MMA per K step, 128 rows of W2;
+//  - down: two MMAs per K step as well, rows 256 f .. +127 and +128 .. +255
+//    of W2 against the same token tile, so each token tile is read once per
+//    256 output features (half the shared-memory and L2 traffic of 128);
 //  - operands arrive by TMA in 128-byte-swizzled K-major boxes of 128 K; E2M1
 //    codes are expanded to one byte per element in shared memory by the
 //    tensor map's 16U4_ALIGN16B type; the E8M0 scales come in 512-byte atoms
@@ -129,7 +131,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     TcSmem &s = tc_smem(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool GU = MODE == kModeGU;
-    const int ft = a.Nw / kTile, kt_n = a.K / kTile;
+    // work items per expert and token tile: 128 gate+up rows (gate/up) or 256
+    // down rows (down), both as two 128-row MMA operands per K step
+    const int ft = a.Nw / (GU ? kTile : 2 * kTile), kt_n = a.K / kTile;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTcStages; ++i) {
@@ -160,23 +164,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             prefetch_tensormap(&a.act);
             // an expanded E2M1 box credits the packed bytes it reads (8 KB), not
             // the 16 KB it fills in shared memory
-            const uint32_t tx = (GU ? 2 : 1) * (kTileBytes / 2) + kTileBytes + (GU ? 3 : 2) * 512;
+            const uint32_t tx = 2 * (kTileBytes / 2) + kTileBytes + 3 * 512;
             int it = 0;
             for (int w = blockIdx.x; w < n_work && !s.abort; w += gridDim.x) {
                 const Work wk = work_of(w, ft, s.ustart, a.E, a.offsets);
-                const int wrow = wk.e * a.Nw + wk.f * kTile;
-                const int64_t wat = ((int64_t)wk.e * ft + wk.f) * kt_n;                    // weight atom base
+                // the two weight tiles: W1 and W3 rows 128 f (gate/up), W2 rows 256 f and 256 f + 128 (down)
+                const int wrow0 = wk.e * a.Nw + wk.f * (GU ? kTile : 2 * kTile), wrow1 = GU ? wrow0 : wrow0 + kTile;
+                const int64_t rg0 = (int64_t)wk.e * (a.Nw / kTile) + (GU ? wk.f : 2 * wk.f);  // 128-row group
+                const int64_t wat0 = rg0 * kt_n, wat1 = (GU ? rg0 : rg0 + 1) * kt_n;        // weight atom bases
                 const int64_t aat = ((int64_t)s.ustart[wk.e] + wk.j) * kt_n;              // activation atom base
                 for (int kt = 0; kt < kt_n; ++kt, ++it) {
                     const int slot = it % kTcStages;
                     if (!mbar_wait(&s.empty[slot], ((it / kTcStages) & 1) ^ 1)) { tc_fail(a, s); break; }
                     uint64_t *bar = &s.full[slot];
                     mbar_arrive_expect_tx(bar, tx);
-                    tma_load_2d(s.a[slot][0], &a.wa, kt * kTile, wrow, bar);
-                    if (GU) tma_load_2d(s.a[slot][1], &a.wb, kt * kTile, wrow, bar);
+                    tma_load_2d(s.a[slot][0], &a.wa, kt * kTile, wrow0, bar);
+                    tma_load_2d(s.a[slot][1], &a.wb, kt * kTile, wrow1, bar);
                     tma_load_2d(s.b[slot], &a.act, kt * kTile, wk.row0, bar);
-                    bulk_g2s(s.sf[slot][0], a.sfa + (wat + kt) * 512, 512, bar);
-                    if (GU) bulk_g2s(s.sf[slot][1], a.sfb + (wat + kt) * 512, 512, bar);
+                    bulk_g2s(s.sf[slot][0], a.sfa + (wat0 + kt) * 512, 512, bar);
+                    bulk_g2s(s.sf[slot][1], a.sfb + (wat1 + kt) * 512, 512, bar);
                     bulk_g2s(s.sf[slot][2], a.sfact + (aat + kt) * 512, 512, bar);
                 }
             }
@@ -201,7 +207,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                     tc_fence_after();
                     const uint32_t sfc = tmem + kSfCol + 16 * slot;
                     tc_cp_sf(sfc, sdesc_sf(s.sf[slot][0]));
-                    if (GU) tc_cp_sf(sfc + 4, sdesc_sf(s.sf[slot][1]));
+                    tc_cp_sf(sfc + 4, sdesc_sf(s.sf[slot][1]));
                     tc_cp_sf(sfc + 8, sdesc_sf(s.sf[slot][2]));
                     const uint64_t d0 = sdesc_sw128(s.a[slot][0]), d1 = sdesc_sw128(s.a[slot][1]),
                                    db = sdesc_sw128(s.b[slot]);
@@ -210,7 +216,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                         const uint32_t id = idesc_sf_ids(idesc, ks, ks), acc = (kt | ks) != 0;
                         const uint32_t sel = (uint32_t)ks << 30;
                         tc_mma_mx(tmem, d0 + 2 * ks, db + 2 * ks, id, sfc | sel, (sfc + 8) | sel, acc);
-                        if (GU) tc_mma_mx(tmem + 128, d1 + 2 * ks, db + 2 * ks, id, (sfc + 4) | sel, (sfc + 8) | sel, acc);
+                        tc_mma_mx(tmem + 128, d1 + 2 * ks, db + 2 * ks, id, (sfc + 4) | sel, (sfc + 8) | sel, acc);
                     }
                     tc_commit(&s.empty[slot]);  // frees the stage once these MMAs finish
                 }
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             // next tile's MMAs overlap the requantisation and the stores.
             const int c0 = 64 * half;
             const int nc = max(0, min(64, wk.nvalid - c0));  // this warp's valid columns
-            float v[64];
+            float v[64], v2[GU ? 1 : 64];  // down: v2 = the second 128 rows
             if (nc > 0) {
                 uint32_t r[32];
 #pragma unroll
@@ -258,9 +264,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                                 v[32 * c + i] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[i]);
                             }
                         } else {
+                            uint32_t r2[32];
+                            tmem_ld32(lane_base + 128 + c0 + 32 * c, r2);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) v[32 * c + i] = __uint_as_float(r[i]);
+                            for (int i = 0; i < 32; ++i) {
+                                v[32 * c + i] = __uint_as_float(r[i]);
+                                if (!GU) v2[32 * c + i] = __uint_as_float(r2[i]);
+                            }
                         }
                     }
                 }
@@ -301,10 +312,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                     }
                 }
             } else {
-                float *orow = a.out + (int64_t)(wk.row0 + c0) * a.Nw + wk.f * kTile + 32 * q + lane;
+                float *orow = a.out + (int64_t)(wk.row0 + c0) * a.Nw + wk.f * 2 * kTile + 32 * q + lane;
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
-                    if (i < nc) orow[(int64_t)i * a.Nw] = v[i];
+                    if (i < nc) {
+                        orow[(int64_t)i * a.Nw] = v[i];
+                        if (!GU) orow[(int64_t)i * a.Nw + kTile] = v2[i];
+                    }
             }
         }
     }
@@ -420,7 +434,7 @@ cudaError_t tc_set_attrs() {
 }  // namespace
 
 bool tc_path_applies(const moe_dims &d) {
-    return d.wfmt == MOE_W_MXFP4 && d.act == MOE_A_MXFP8 && d.d_model % kTile == 0 && d.d_ff % kTile == 0 &&
+    return d.wfmt == MOE_W_MXFP4 && d.act == MOE_A_MXFP8 && d.d_model % (2 * kTile) == 0 && d.d_ff % kTile == 0 &&
            d.E <= kTcMaxE && d.T >= 1;
 }
 
@@ -447,12 +461,13 @@ cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_
     TcArgs dn;
     memset(&dn, 0, sizeof dn);
     ok = ok && make_tile_map_e2m1(&dn.wa, p2 + L2.codes, r2, d.d_ff, kTile) &&
+         make_tile_map_e2m1(&dn.wb, p2 + L2.codes, r2, d.d_ff, kTile) &&
          make_tile_map_u8(&dn.act, h8, S, d.d_ff, kTile);
     if (!ok) return cudaErrorInvalidValue;
     g.sfa = p1 + L1.stile; g.sfb = p3 + L1.stile; g.sfact = gxsf;
     g.offsets = offsets; g.ustart = ustart; g.E = d.E; g.Nw = d.d_ff; g.K = d.d_model;
     g.h8 = h8; g.hsf = hsf; g.err = device_error_word();
-    dn.sfa = p2 + L2.stile; dn.sfact = hsf;
+    dn.sfa = p2 + L2.stile; dn.sfb = p2 + L2.stile; dn.sfact = hsf;
     dn.offsets = offsets; dn.ustart = ustart; dn.E = d.E; dn.Nw = d.d_model; dn.K = d.d_ff;
     dn.out = out_rows; dn.err = g.err;
 
