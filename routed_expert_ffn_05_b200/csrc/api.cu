@@ -28,10 +28,12 @@ static cudaEvent_t g_ffn_before = nullptr, g_ffn_after = nullptr;
 // Routed-expert FFN bracketed by the optional profiling events.
 static cudaError_t expert_ffn_timed(const moe_dims &d, const moe_weights &w, const uint16_t *x,
                                     const int32_t *offsets, const int32_t *perm, float *rows, float *shared,
-                                    uint8_t *ws, const WsLayout &L, cudaStream_t s, bool prepared = false) {
+                                    uint8_t *ws, const WsLayout &L, cudaStream_t s, bool prepared = false,
+                                    bool rows_bf16 = false) {
     cudaError_t e;
     if (g_ffn_before && g_ffn_after && (e = cudaEventRecord(g_ffn_before, s)) != cudaSuccess) return e;
-    if ((e = launch_expert_ffn(d, w, x, offsets, perm, rows, shared, ws, L, s, prepared)) != cudaSuccess) return e;
+    if ((e = launch_expert_ffn(d, w, x, offsets, perm, rows, shared, ws, L, s, prepared, rows_bf16)) != cudaSuccess)
+        return e;
     if (g_ffn_before && g_ffn_after) return cudaEventRecord(g_ffn_after, s);
     return cudaSuccess;
 }
@@ -233,7 +235,11 @@ moe_status moe_layer(const moe_dims *dims, const moe_weights *weights, const uin
                                 reinterpret_cast<int32_t *>(w + L.blkbase), L.nblk, s)))
             return cuda_status(e);
     }
-    if ((e = expert_ffn_timed(d, *weights, x, offsets, perm, rows, sh, w, L, s, fused))) return cuda_status(e);
+    // the tensor-core path hands its rows to the combine as bf16 (half the traffic)
+    const bool r16 = tc_path_applies(d);
+    if ((e = expert_ffn_timed(d, *weights, x, offsets, perm, rows, sh, w, L, s, fused, r16))) return cuda_status(e);
+    if (r16)
+        return cuda_status(launch_combine_bf16(d, reinterpret_cast<const uint16_t *>(rows), inv, gates, sh, y, s));
     return cuda_status(launch_combine(d, rows, inv, gates, sh, y, s, decode_path_applies(d)));
 }
 

@@ -1,12 +1,22 @@
 // Gate-weighted combine: y[t] = sum_{j ascending} w[t,j] * o[inv_perm[t*k+j]]
-// (+ shared expert s[t]), fp32, the k terms in a fixed order.
+// (+ shared expert s[t]), fp32, the k terms in a fixed order. The expert
+// rows o are fp32 (the staged API) or bf16 (the fused layer's w4a8 path,
+// which halves their write and read traffic).
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace moe {
 
-__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ out_rows,
+__device__ __forceinline__ float4 load_row4(const float *r, int i4) { return reinterpret_cast<const float4 *>(r)[i4]; }
+__device__ __forceinline__ float4 load_row4(const uint16_t *r, int i4) {
+    const uint2 v = reinterpret_cast<const uint2 *>(r)[i4];
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                       __uint_as_float(v.y & 0xFFFF0000u));
+}
+
+template <typename R>
+__global__ void __launch_bounds__(256) combine_kernel(const R *__restrict__ out_rows,
                                                       const int32_t *__restrict__ inv_perm,
                                                       const float *__restrict__ gates,
                                                       const float *__restrict__ shared, int d, int k,
@@ -21,7 +31,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     for (int j = 0; j < k; ++j) {
         const int64_t s = (int64_t)t * k + j;
         const float g = gates[s];
-        const float4 o = reinterpret_cast<const float4 *>(out_rows + (int64_t)inv_perm[s] * d)[i4];
+        const float4 o = load_row4(out_rows + (int64_t)inv_perm[s] * d, i4);
         sum.x = fmaf(g, o.x, sum.x);
         sum.y = fmaf(g, o.y, sum.y);
         sum.z = fmaf(g, o.z, sum.z);
@@ -34,8 +44,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     reinterpret_cast<float4 *>(y + (int64_t)t * d)[i4] = acc;
 }
 
-cudaError_t launch_combine(const moe_dims &d, const float *out_rows, const int32_t *inv_perm,
-                           const float *gates, const float *shared, float *y, cudaStream_t s, bool pdl) {
+template <typename R>
+static cudaError_t launch_combine_t(const moe_dims &d, const R *out_rows, const int32_t *inv_perm,
+                                   const float *gates, const float *shared, float *y, cudaStream_t s, bool pdl) {
     if (d.T == 0) return cudaSuccess;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -47,9 +58,19 @@ cudaError_t launch_combine(const moe_dims &d, const float *out_rows, const int32
     cfg.attrs = pdl ? attr : nullptr;
     cfg.numAttrs = pdl ? 1 : 0;
     const int dm = d.d_model, k = d.k;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, out_rows, inv_perm, gates, shared, dm, k, y);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel<R>, out_rows, inv_perm, gates, shared, dm, k, y);
     count_launches(1);
     return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_combine(const moe_dims &d, const float *out_rows, const int32_t *inv_perm,
+                           const float *gates, const float *shared, float *y, cudaStream_t s, bool pdl) {
+    return launch_combine_t(d, out_rows, inv_perm, gates, shared, y, s, pdl);
+}
+
+cudaError_t launch_combine_bf16(const moe_dims &d, const uint16_t *out_rows, const int32_t *inv_perm,
+                                const float *gates, const float *shared, float *y, cudaStream_t s) {
+    return launch_combine_t(d, out_rows, inv_perm, gates, shared, y, s, false);
 }
 
 }  // namespace moe

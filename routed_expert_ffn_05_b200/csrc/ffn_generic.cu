@@ -187,14 +187,14 @@ cudaError_t launch_shared_ffn_generic(const moe_dims &d, const moe_weights &w, c
 
 cudaError_t launch_expert_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x,
                               const int32_t *offsets, const int32_t *perm, float *out_rows, float *shared_out,
-                              uint8_t *ws, const WsLayout &L, cudaStream_t s, bool prepared) {
+                              uint8_t *ws, const WsLayout &L, cudaStream_t s, bool prepared, bool rows_bf16) {
     if (decode_path_applies(d))
         return launch_decode_ffn(d, w, x, offsets, perm, out_rows, shared_out, ws, L, s, prepared);
     cudaError_t e;
     if (shared_out &&
         (e = launch_shared_ffn_generic(d, w, x, shared_out, reinterpret_cast<float *>(ws + L.sh_h), s)) != cudaSuccess)
         return e;
-    if (tc_path_applies(d)) return launch_tc_ffn(d, w, x, offsets, perm, out_rows, ws, L, s);
+    if (tc_path_applies(d)) return launch_tc_ffn(d, w, x, offsets, perm, out_rows, ws, L, s, rows_bf16);
     return launch_expert_ffn_generic(d, w, x, offsets, perm, out_rows, ws, L, s);
 }
 

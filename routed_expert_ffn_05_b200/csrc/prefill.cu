@@ -56,7 +56,8 @@ struct TcArgs {
     int E, Nw, K;              // weight rows per expert, K
     uint8_t *h8;               // gate/up: h codes [S][F]
     uint8_t *hsf;              // gate/up: h scale atoms [tiles][F/128][512]
-    float *out;                // down: rows [S][d]
+    float *out;                // down: rows [S][d] fp32, or
+    uint16_t *out16;           //       bf16 when this is set
     int *err;
 };
 
@@ -312,13 +313,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                     }
                 }
             } else {
-                float *orow = a.out + (int64_t)(wk.row0 + c0) * a.Nw + wk.f * 2 * kTile + 32 * q + lane;
+                const int64_t o0 = (int64_t)(wk.row0 + c0) * a.Nw + wk.f * 2 * kTile + 32 * q + lane;
+                if (a.out16) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (i < nc) {
-                        orow[(int64_t)i * a.Nw] = v[i];
-                        if (!GU) orow[(int64_t)i * a.Nw + kTile] = v2[i];
-                    }
+                    for (int i = 0; i < 64; ++i)
+                        if (i < nc) {
+                            a.out16[o0 + (int64_t)i * a.Nw] = f32_to_bf16_rne(v[i]);
+                            if (!GU) a.out16[o0 + (int64_t)i * a.Nw + kTile] = f32_to_bf16_rne(v2[i]);
+                        }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (i < nc) {
+                            a.out[o0 + (int64_t)i * a.Nw] = v[i];
+                            if (!GU) a.out[o0 + (int64_t)i * a.Nw + kTile] = v2[i];
+                        }
+                }
             }
         }
     }
@@ -441,7 +451,8 @@ bool tc_path_applies(const moe_dims &d) {
 // Routed expert FFN (w4a8, MXFP4 weights) on the tensor cores: plan, gather +
 // quantise, gate/up GEMM with SwiGLU and MXFP8 requantisation, down GEMM.
 cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
-                          const int32_t *perm, float *out_rows, uint8_t *ws, const WsLayout &L, cudaStream_t s) {
+                          const int32_t *perm, float *out_rows, uint8_t *ws, const WsLayout &L, cudaStream_t s,
+                          bool rows_bf16) {
     const int S = d.T * d.k;
     if (S == 0) return cudaSuccess;
     cudaError_t e = tc_set_attrs();
@@ -469,7 +480,9 @@ cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_
     g.h8 = h8; g.hsf = hsf; g.err = device_error_word();
     dn.sfa = p2 + L2.stile; dn.sfb = p2 + L2.stile; dn.sfact = hsf;
     dn.offsets = offsets; dn.ustart = ustart; dn.E = d.E; dn.Nw = d.d_model; dn.K = d.d_ff;
-    dn.out = out_rows; dn.err = g.err;
+    if (rows_bf16) dn.out16 = reinterpret_cast<uint16_t *>(out_rows);
+    else dn.out = out_rows;
+    dn.err = g.err;
 
     tc_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, ustart);
     tc_gather_quant_kernel<<<(S + 7) / 8, 256, 0, s>>>(x, offsets, perm, ustart, S, d.E, d.k, d.d_model, gx8, gxsf);
