@@ -174,12 +174,12 @@ def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=
         a.record(stream)
         b.record(stream)
 
-    def step(i, timed):
+    def step(i, timed, ffn_events=False):
         b = i % batches
         flush.fill_(i & 0xFF)
         if timed:
             ev[i][0].record(stream)
-            if not e2e:
+            if ffn_events:
                 M.moe_debug_set_ffn_events(fev[i][0], fev[i][1])
         if e2e:
             xd.copy_(xh[b], non_blocking=True)
@@ -190,7 +190,7 @@ def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=
         else:
             M.moe_layer(dims, layer.weights, xs[b], toks[b], y, ws)
         if timed:
-            if not e2e:
+            if ffn_events:
                 M.moe_debug_set_ffn_events(None, None)
             ev[i][1].record(stream)
 
@@ -209,7 +209,20 @@ def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=
     times = [a.elapsed_time(b) for a, b in ev]
     out = {"ms": times, "launches": n1 - n0}
     if not e2e:
+        # A second pass with the library's FFN events installed times the expert
+        # FFN stage alone (for the roofline). The events split the launch chain
+        # (no early start of the FFN kernel during routing), so the layer time
+        # above comes from the first, uninstrumented pass.
+        barrier(torch, world)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            step(i, True, ffn_events=True)
+        torch.cuda.synchronize()
+        barrier(torch, world)
+        if M.moe_get_device_error() != 0:
+            raise RuntimeError("device error word set during the benchmark")
         out["ffn_ms"] = [a.elapsed_time(b) for a, b in fev]
+        out["ms_with_ffn_events"] = [a.elapsed_time(b) for a, b in ev]
     return out
 
 

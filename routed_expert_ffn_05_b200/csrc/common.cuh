@@ -66,6 +66,50 @@ __device__ __forceinline__ int expert_of_row(const int32_t *offsets, int E, int 
     return lo;
 }
 
+// Ranking key of (logit v, expert e): keys compare as unsigned integers in
+// the routing order -- larger logit first, NaN after every number, ties (and
+// +0 == -0) by the lower expert index. High word: the float made monotone
+// (-0 as +0, NaN as 0); low word: ~e. Key 0 is below every valid key.
+__device__ __forceinline__ uint64_t rank_key(float v, int e) {
+    uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    u = isnan(v) ? 0u : u;
+    return ((uint64_t)u << 32) | (uint32_t)~(uint32_t)e;
+}
+__device__ __forceinline__ int rank_key_expert(uint64_t key) { return (int)~(uint32_t)key; }
+
+// Warp-wide top-k of one row of E <= 1024 logits: lane holds cv[i] = logit of
+// expert lane + 32 i (i < ceil(E / 32)). Round j takes the warp maximum of the
+// unchosen keys; lane j receives pick j in my_e. Callers read the picked
+// logits back by expert index.
+__device__ __forceinline__ int topk_warp(const float (&cv)[32], int E, int k, int lane) {
+    const int nc = (E + 31) >> 5;
+    uint64_t key[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) key[i] = (i < nc && lane + 32 * i < E) ? rank_key(cv[i], lane + 32 * i) : 0ull;
+    int my_e = -1;
+    for (int j = 0; j < k; ++j) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i >= nc) break;  // uniform
+            best = key[i] > best ? key[i] : best;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i >= nc) break;
+            key[i] = key[i] == best ? 0ull : key[i];  // keys are unique: only the pick matches
+        }
+        my_e = lane == j ? rank_key_expert(best) : my_e;
+    }
+    return my_e;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -40,6 +40,17 @@
 #include "ptx.cuh"
 #include "tma.h"
 
+__device__ unsigned long long g_st[16];
+#define STMIN(i) atomicMin(&g_st[i], (unsigned long long)moe::globaltimer_ns())
+#define STMAX(i) atomicMax(&g_st[i], (unsigned long long)moe::globaltimer_ns())
+extern "C" __attribute__((visibility("default"))) int moe_dbg_stamps(unsigned long long *h, int reset) {
+    if (reset) {
+        unsigned long long v[16];
+        for (int i = 0; i < 16; ++i) v[i] = (i % 2 == 0 && i < 10) ? ~0ull : 0ull;
+        return (int)cudaMemcpyToSymbol(g_st, v, sizeof v);
+    }
+    return (int)cudaMemcpyFromSymbol(h, g_st, sizeof(unsigned long long) * 16);
+}
 namespace moe {
 namespace {
 
@@ -114,6 +125,31 @@ __device__ __forceinline__ int sigma(int g) { return (g >> 1) | ((g & 1) << 2); 
 struct Unit {
     int kind, seg, tile, nst;
 };
+
+// Warp-wide: the experts with rows (offsets[e + 1] > offsets[e]) in ascending
+// order; f(segment, expert, first row, end row) runs on the lane that found
+// each one. Loads 8 x 32 experts' offsets at a time. Returns the count.
+template <typename F>
+__device__ __forceinline__ int active_experts(const int32_t *offsets, int E, int lane, F f) {
+    int n = 0;
+    for (int b0 = 0; b0 < E; b0 += 256) {
+        int lo[8], hi[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = b0 + 32 * j + lane;
+            lo[j] = e < E ? __ldcg(&offsets[e]) : 0;
+            hi[j] = e < E ? __ldcg(&offsets[e + 1]) : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const bool act = hi[j] > lo[j];
+            const unsigned m = __ballot_sync(0xffffffffu, act);
+            if (act) f(n + __popc(m & ((1u << lane) - 1u)), b0 + 32 * j + lane, lo[j], hi[j]);
+            n += __popc(m);
+        }
+    }
+    return n;
+}
 
 // Unit numbering: [shared gate/up][routed gate/up][shared down][routed down].
 // Shared gate/up units are assigned statically (they need no routing), routed
@@ -339,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     extern __shared__ uint8_t smem_raw[];
     Smem &s = smem_ref(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) STMIN(4);
     if (threadIdx.x == kProducer * 32) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&s.full[i], 1);
@@ -419,14 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         }
         __syncwarp();
         grid_dep_wait();  // routing results and zeroed counters from here on
-        int n = 0;        // active experts, ascending
-        for (int e0 = 0; e0 < a.E; e0 += 32) {
-            const int e = e0 + lane;
-            const bool act = e < a.E && a.offsets[e + 1] > a.offsets[e];
-            const unsigned m = __ballot_sync(0xffffffffu, act);
-            if (act) s.seg_e[n + __popc(m & ((1u << lane) - 1u))] = e;
-            n += __popc(m);
-        }
+        const int n = active_experts(a.offsets, a.E, lane, [&](int sg, int e, int, int) { s.seg_e[sg] = e; });
         if (lane != 0) return;
         s.n_seg = n;
         const int gu_end = usg + n * kGuTiles;
@@ -480,21 +510,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     if (warp == kEpilogue) {
         grid_dep_wait();
         // per-expert tables, same ascending order as the producer's list
-        int n = 0;
-        for (int e0 = 0; e0 < a.E; e0 += 32) {
-            const int e = e0 + lane;
-            const bool act = e < a.E && a.offsets[e + 1] > a.offsets[e];
-            const unsigned m = __ballot_sync(0xffffffffu, act);
-            if (act) {
-                const int sg = n + __popc(m & ((1u << lane) - 1u));
-                s.ep_rbase[sg] = a.offsets[e];
-                s.ep_cnt[sg] = (uint8_t)(a.offsets[e + 1] - a.offsets[e]);
-            }
-            n += __popc(m);
-        }
+        const int n = active_experts(a.offsets, a.E, lane, [&](int sg, int, int r0, int r1) {
+            s.ep_rbase[sg] = r0;
+            s.ep_cnt[sg] = (uint8_t)(r1 - r0);
+        });
         __syncwarp();
-        for (int sg = lane; sg < n; sg += 32)
-            for (int i = 0; i < s.ep_cnt[sg]; ++i) s.ep_tok[sg][i] = (uint8_t)(a.perm[s.ep_rbase[sg] + i] / a.k);
+        for (int sg = lane; sg < n; sg += 32) {
+            const int rb = s.ep_rbase[sg], cnt = s.ep_cnt[sg];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i < cnt) s.ep_tok[sg][i] = (uint8_t)(__ldcg(&a.perm[rb + i]) / a.k);
+        }
         if (lane < a.T) s.ep_xs[lane] = a.xscale[lane].x;
         __syncwarp();
         // gate/up tiles finished here and not yet published: shared, and routed of segment pseg
@@ -614,6 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     int bkind = -1, bseg = -2;  // what B holds
     bool dep = false;           // grid dependency resolved for this thread
     bool flushed = false;       // gate/up count of this CTA published
+    bool dphase = false;
     float acc[2][4];
     int ru = 0;
     auto marker = [&](int m) {  // a hand-off without a tile: -1 end, -2 publish
@@ -628,13 +655,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         const int slot = gi % kStages;
         if (!mbar_wait(&s.full[slot], (gi / kStages) & 1)) { fail(a, s); return; }
         const int u = s.meta_u[slot], c = s.meta_c[slot];
+        if (u < 0 && threadIdx.x == 0) STMAX(11);
         if (u < 0) {  // end of work: publish (if still due) and tell the epilogue
             if ((!flushed && !marker(-2)) || !marker(-1)) fail(a, s);
             return;
         }
         const Unit un = unit_of<WF>(u, usg, u < usg ? 0 : s.n_seg, usd);
+        if ((un.kind == kDsh || un.kind == kDrt) && !dphase) { dphase = true; if (threadIdx.x == 0) { STMIN(8); STMAX(13); } }
         if (un.kind != kGsh && !dep) {
             grid_dep_wait();
+            if (threadIdx.x == 0) { STMIN(6); STMAX(9); }
             dep = true;
         }
         // B depends on the kind, and for down units on the expert (its h rows)
@@ -771,77 +801,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 }
 
 // ---------------------------------------------------------------------------
-// Decode routing: fixed-order fp32 logits (one warp per expert, lane = chunk,
-// all T tokens at once; CTA 0 also computes the per-token f16 prescale), then
+// Decode routing: fixed-order fp32 logits (one CTA per expert, one warp per
+// token, lane = chunk; CTA 0 also computes the per-token f16 prescale), then
 // one CTA does top-k, softmax gates, histogram / scan / permutation and
 // resets the FFN kernel's scratch.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int xs_index(int t, int c, int v) { return (t * 32 + c) * 17 + v; }  // padded [T][32][17] uint4
-
-__global__ void __launch_bounds__(128) decode_logits_kernel(const uint16_t *__restrict__ x,
+// One CTA per expert, one warp per token: lane c runs the fma chain over
+// chunk c (elements 128 c .. 128 c + 127) in element order, then the fixed
+// butterfly across the chunks. The expert's router row is staged once per CTA
+// in shared memory as [16][32 lanes] uint4; the token's x chunk stays in
+// registers. The warps of CTA 0 also write the per-token x prescale.
+__global__ void __launch_bounds__(256) decode_logits_kernel(const uint16_t *__restrict__ x,
                                                             const uint16_t *__restrict__ wr,
                                                             const float *__restrict__ bias, int T, int E,
                                                             float *__restrict__ logits, float2 *__restrict__ xscale) {
-    extern __shared__ uint4 xs4[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 4 + warp;
+    __shared__ uint4 ws4[16 * 32];
+    const int t = threadIdx.x >> 5, lane = threadIdx.x & 31, e = blockIdx.x;
+    if (threadIdx.x == 0) STMIN(0);
     constexpr int chunk = kD / 32;  // 128 elements = 16 uint4 per lane
-    uint4 wv[16];
-    if (e < E)
+    for (int i = threadIdx.x; i < 16 * 32; i += blockDim.x)
+        cp_async_16(&ws4[i], wr + (int64_t)e * kD + (i & 31) * chunk + 8 * (i >> 5));
+    uint4 xv[16];
 #pragma unroll
-        for (int v = 0; v < 16; ++v) wv[v] = ldg128(wr + (int64_t)e * kD + lane * chunk + 8 * v);
-    for (int i = threadIdx.x; i < T * 512; i += blockDim.x) xs4[xs_index(i / 512, (i / 16) % 32, i % 16)] = ldg128(x + 8 * i);
+    for (int v = 0; v < 16; ++v) xv[v] = ldg128(x + (int64_t)t * kD + lane * chunk + 8 * v);
+    cp_async_wait_all();
     __syncthreads();
+    if (threadIdx.x == 0) STMAX(1);
     grid_dep_launch();
-    if (blockIdx.x == 0)
-        for (int t = warp; t < T; t += 4) {  // per-token 2^p with max|x| 2^-p in [2^14, 2^15)
-            float mx = 0.f;
-            for (int i = lane; i < 512; i += 32) {
-                const uint4 v = xs4[xs_index(t, i / 16, i % 16)];
-                const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+    if (e == 0) {  // 2^p with max|x_t| 2^-p in [2^14, 2^15)
+        float mx = 0.f;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(r[j] << 16)), fabsf(__uint_as_float(r[j] & 0xFFFF0000u))));
-            }
+        for (int v = 0; v < 16; ++v) {
+            const uint32_t r[4] = {xv[v].x, xv[v].y, xv[v].z, xv[v].w};
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (lane == 0) {
-                const int p = mx > 0.f ? floor_log2_f32(mx) - 14 : 0;
-                xscale[t] = make_float2(ldexpf(1.0f, p), ldexpf(1.0f, -p));
-            }
+            for (int j = 0; j < 4; ++j)
+                mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(r[j] << 16)), fabsf(__uint_as_float(r[j] & 0xFFFF0000u))));
         }
-    if (e >= E) return;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) {
+            const int p = mx > 0.f ? floor_log2_f32(mx) - 14 : 0;
+            xscale[t] = make_float2(ldexpf(1.0f, p), ldexpf(1.0f, -p));
+        }
+    }
+    float acc = 0.f;
 #pragma unroll
     for (int v = 0; v < 16; ++v) {
-        const uint32_t wa[4] = {wv[v].x, wv[v].y, wv[v].z, wv[v].w};
+        const uint4 wq = ws4[v * 32 + lane];
+        const uint32_t wa[4] = {wq.x, wq.y, wq.z, wq.w};
+        const uint32_t xa[4] = {xv[v].x, xv[v].y, xv[v].z, xv[v].w};
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
-            if (t < T) {
-                const uint4 xv = xs4[xs_index(t, lane, v)];
-                const uint32_t xa[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    acc[t] = __fmaf_rn(__uint_as_float(xa[qq] << 16), __uint_as_float(wa[qq] << 16), acc[t]);
-                    acc[t] = __fmaf_rn(__uint_as_float(xa[qq] & 0xFFFF0000u), __uint_as_float(wa[qq] & 0xFFFF0000u), acc[t]);
-                }
-            }
+        for (int qq = 0; qq < 4; ++qq) {
+            acc = __fmaf_rn(__uint_as_float(xa[qq] << 16), __uint_as_float(wa[qq] << 16), acc);
+            acc = __fmaf_rn(__uint_as_float(xa[qq] & 0xFFFF0000u), __uint_as_float(wa[qq] & 0xFFFF0000u), acc);
+        }
     }
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
-        if (t < T) {
-            float v = acc[t];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
-            if (lane == 0) logits[(int64_t)t * E + e] = bias ? __fadd_rn(v, bias[e]) : v;
-        }
-}
-
-__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
-    const bool na = isnan(va), nb = isnan(vb);
-    if (na != nb) return nb;
-    if (!na && va != vb) return va > vb;
-    return ia < ib;
+    for (int o = 1; o < 32; o <<= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+    if (lane == 0) logits[(int64_t)t * E + e] = bias ? __fadd_rn(acc, bias[e]) : acc;
+    if (lane == 0) STMAX(3);
 }
 
 struct FinalizeArgs {
@@ -856,38 +874,39 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
     __shared__ float lg[8 * kMaxE];
     __shared__ int hist[kMaxE];
     __shared__ int sidx[256];
+    __shared__ int run[kMaxE];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, E = a.E, k = a.k;
     grid_dep_launch();
     for (int i = threadIdx.x; i < E + 2; i += blockDim.x) a.counters[i] = 0u;
     for (int i = threadIdx.x; i < T * k; i += blockDim.x) a.hmax[i] = 0u;
+    if (threadIdx.x == 0) STMIN(2);
     grid_dep_wait();
-    for (int i = threadIdx.x; i < T * E; i += blockDim.x) lg[i] = a.logits[i];
-    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-    __syncthreads();
-    if (warp < T) {  // top-k + gates of token `warp`
-        const float *l = lg + warp * E;
-        uint32_t taken = 0;
-        float my_l = 0.f, l0v = 0.f;
-        int my_e = -1;
-        for (int j = 0; j < k; ++j) {
-            float bv = 0.f;
-            int bi = -1;
-            for (int i = 0, e = lane; e < E; ++i, e += 32) {
-                if (taken >> i & 1u) continue;
-                const float v = l[e];
-                if (bi < 0 || ranks_before(v, e, bv, bi)) { bv = v; bi = e; }
-            }
+    if (threadIdx.x == 0) STMAX(5);
+    for (int base = 0; base < T * E; base += 8 * 256) {  // 8 loads in flight per thread
+        float v[8];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (oi >= 0 && (bi < 0 || ranks_before(ov, oi, bv, bi))) { bv = ov; bi = oi; }
-            }
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-            if (j == 0) l0v = bv;
-            if (lane == j) { my_l = bv; my_e = bi; }
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + 256 * j + threadIdx.x;
+            v[j] = i < T * E ? __ldcg(a.logits + i) : 0.f;
         }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + 256 * j + threadIdx.x;
+            if (i < T * E) lg[i] = v[j];
+        }
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = run[e] = 0;
+    __syncthreads();
+    if (threadIdx.x == 0) STMAX(10);
+    if (warp < T) {  // top-k + gates of token `warp`: lane holds experts lane + 32 i
+        const float *l = lg + warp * E;
+        float cv[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) cv[i] = lane + 32 * i < E ? l[lane + 32 * i] : 0.f;
+        const int my_e = topk_warp(cv, E, k, lane);
+        const float my_l = lane < k ? l[my_e] : 0.f;
+        const float l0v = __shfl_sync(0xffffffffu, my_l, 0);
         const float ex = lane < k ? expf(my_l - l0v) : 0.f;
         const float den = warp_sum(ex);
         if (lane < k) {
@@ -897,38 +916,51 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
         }
     }
     __syncthreads();
+    if (threadIdx.x == 0) STMAX(12);
     const int S = T * k;
     if (threadIdx.x < S) atomicAdd(&hist[sidx[threadIdx.x]], 1);
     __syncthreads();
-    if (warp == 0) {  // exclusive scan over experts
-        int run = 0;
-        for (int e0 = 0; e0 < E; e0 += 32) {
-            const int e = e0 + lane;
-            const int c = e < E ? hist[e] : 0;
-            int incl = c;
+    if (warp == 0) {  // exclusive scan over experts; lane owns experts [lane * per, (lane + 1) * per)
+        const int per = (E + 31) / 32, e0 = lane * per, e1 = min(E, e0 + per);
+        int tot = 0;
+        for (int e = e0; e < e1; ++e) tot += hist[e];
+        int incl = tot;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            if (e < E) {
-                a.counts[e] = c;
-                a.offsets[e] = run + incl - c;
-                hist[e] = run + incl - c;  // first row of expert e
-            }
-            run += __shfl_sync(0xffffffffu, incl, 31);
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        if (lane == 0) a.offsets[E] = run;
+        int off = incl - tot;
+        for (int e = e0; e < e1; ++e) {
+            const int c = hist[e];
+            a.counts[e] = c;
+            a.offsets[e] = off;
+            hist[e] = off;  // first row of expert e
+            off += c;
+        }
+        if (lane == 31) a.offsets[E] = incl;
     }
     __syncthreads();
-    if (threadIdx.x < S) {  // stable rank: earlier slots of the same expert
-        const int s0 = threadIdx.x, e = sidx[s0];
-        int r = 0;
-        for (int s1 = 0; s1 < s0; ++s1) r += (sidx[s1] == e);
-        const int row = hist[e] + r;
-        a.perm[row] = s0;
-        a.inv_perm[s0] = row;
+    if (threadIdx.x == 0) STMAX(14);
+    // stable rank of each slot among the earlier slots of its expert: within a
+    // warp by matching lanes, across warps through a running count per expert
+    for (int w0 = 0; w0 * 32 < S; ++w0) {
+        if (warp == w0) {
+            const int s0 = threadIdx.x;
+            const bool in = s0 < S;
+            const int e = in ? sidx[s0] : -1 - lane;
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            if (in) {
+                const int row = hist[e] + run[e] + __popc(peers & ((1u << lane) - 1u));
+                a.perm[row] = s0;
+                a.inv_perm[s0] = row;
+            }
+            __syncwarp();
+            if (in && lane == 31 - __clz(peers)) run[e] += __popc(peers);
+        }
+        __syncthreads();
     }
+    if (threadIdx.x == 0) STMAX(7);
 }
 
 // Stage-API entry (no routing in this call): the x prescale and the scratch reset.
@@ -961,8 +993,6 @@ int num_sms() {
     return n;
 }
 
-constexpr int kLogitsSmem = 8 * 32 * 17 * 16;
-
 cudaError_t set_smem_attrs() {
     static bool done[64] = {false};
     int dev = 0;
@@ -974,8 +1004,6 @@ cudaError_t set_smem_attrs() {
         return e;
     if ((e = cudaFuncSetAttribute(decode_ffn_kernel<MOE_W_Q2K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kSmemBytes)))
-        return e;
-    if ((e = cudaFuncSetAttribute(decode_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLogitsSmem)))
         return e;
     done[dev] = true;
     return cudaSuccess;
@@ -1020,8 +1048,8 @@ cudaError_t launch_decode_route(const moe_dims &d, const uint16_t *x, const moe_
     cudaError_t e = set_smem_attrs();
     if (e != cudaSuccess) return e;
     float *logits = reinterpret_cast<float *>(ws + L.logits);
-    decode_logits_kernel<<<ceil_div(d.E, 4), 128, kLogitsSmem, s>>>(x, w.w_router, w.router_bias, d.T, d.E, logits,
-                                                                    reinterpret_cast<float2 *>(ws + L.xscale));
+    decode_logits_kernel<<<d.E, 32 * d.T, 0, s>>>(x, w.w_router, w.router_bias, d.T, d.E, logits,
+                                                  reinterpret_cast<float2 *>(ws + L.xscale));
     FinalizeArgs f;
     f.T = d.T; f.E = d.E; f.k = d.k; f.logits = logits;
     f.idx = idx; f.counts = counts; f.offsets = offsets; f.perm = perm; f.inv_perm = inv_perm; f.gates = gates;

@@ -105,6 +105,13 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
 }
 __device__ __forceinline__ uint4 ldcg128(const void *p) { return __ldcg(reinterpret_cast<const uint4 *>(p)); }
 
+// Asynchronous global -> shared copies (LDGSTS): many can be in flight per
+// thread without holding registers. 16-byte copies bypass L1.
+__device__ __forceinline__ void cp_async_16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Byte offset of 16-byte unit u of row r inside a box written by a chunked,
 // 128-byte-swizzled tensor map with `rows` rows per chunk (see tma.h).
 __device__ __forceinline__ int swz_off(int chunk, int rows, int r, int u) {

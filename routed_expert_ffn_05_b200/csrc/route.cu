@@ -155,15 +155,6 @@ __global__ void __launch_bounds__(256, 1) router_tiled_kernel(const uint16_t *__
         }
 }
 
-// a ranks before b: larger logit first, NaN after every number, ties (and
-// +0 == -0) by the lower index.
-__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
-    const bool na = isnan(va), nb = isnan(vb);
-    if (na != nb) return nb;
-    if (!na && va != vb) return va > vb;
-    return ia < ib;
-}
-
 // One warp per token: k rounds of a warp arg-max over the unchosen experts,
 // then the softmax of the k chosen logits.
 __global__ void __launch_bounds__(256) topk_softmax_kernel(const float *__restrict__ logits, int T,
@@ -172,28 +163,12 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float *__restri
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (t >= T) return;
     const float *l = logits + (int64_t)t * E;
-    uint32_t taken = 0;  // bit i: expert lane + 32 i chosen (E <= 1024)
-    float my_l = 0.0f;
-    int my_e = -1;
-    float l0 = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        float bv = 0.0f;
-        int bi = -1;
-        for (int i = 0, e = lane; e < E; ++i, e += 32) {
-            if (taken >> i & 1u) continue;
-            const float v = l[e];
-            if (bi < 0 || ranks_before(v, e, bv, bi)) { bv = v; bi = e; }
-        }
+    float cv[32];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (oi >= 0 && (bi < 0 || ranks_before(ov, oi, bv, bi))) { bv = ov; bi = oi; }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (j == 0) l0 = bv;
-        if (lane == j) { my_l = bv; my_e = bi; }
-    }
+    for (int i = 0; i < 32; ++i) cv[i] = lane + 32 * i < E ? l[lane + 32 * i] : 0.f;
+    const int my_e = topk_warp(cv, E, k, lane);
+    const float my_l = lane < k ? l[my_e] : 0.f;
+    const float l0 = __shfl_sync(0xffffffffu, my_l, 0);
     const float ex = lane < k ? expf(my_l - l0) : 0.0f;
     const float den = warp_sum(ex);
     if (lane < k) {
