@@ -40,17 +40,6 @@
 #include "ptx.cuh"
 #include "tma.h"
 
-__device__ unsigned long long g_st[16];
-#define STMIN(i) atomicMin(&g_st[i], (unsigned long long)moe::globaltimer_ns())
-#define STMAX(i) atomicMax(&g_st[i], (unsigned long long)moe::globaltimer_ns())
-extern "C" __attribute__((visibility("default"))) int moe_dbg_stamps(unsigned long long *h, int reset) {
-    if (reset) {
-        unsigned long long v[16];
-        for (int i = 0; i < 16; ++i) v[i] = (i % 2 == 0 && i < 10) ? ~0ull : 0ull;
-        return (int)cudaMemcpyToSymbol(g_st, v, sizeof v);
-    }
-    return (int)cudaMemcpyFromSymbol(h, g_st, sizeof(unsigned long long) * 16);
-}
 namespace moe {
 namespace {
 
@@ -235,6 +224,10 @@ __device__ __forceinline__ void put_partial(float *r, int rg, int q, const float
     r[(rg + 8) * 8 + 2 * q + 1] = acc[3];
 }
 
+// Byte offset of scale word w (the E8M0 bytes of 32-blocks 4w .. 4w + 3) of
+// row r in a 64-byte-swizzled scale box (rows of 64 bytes).
+__device__ __forceinline__ int scale_off(int r, int w) { return r * 64 + ((((w >> 2) ^ (r >> 1)) & 3) << 4) + 4 * (w & 3); }
+
 // bf16 pair -> f16 pair scaled by an exact power of two.
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v, float sc) {
     return f32x2_to_f16x2(__uint_as_float(v << 16) * sc, __uint_as_float(v & 0xFFFF0000u) * sc);
@@ -375,7 +368,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     extern __shared__ uint8_t smem_raw[];
     Smem &s = smem_ref(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) STMIN(4);
     if (threadIdx.x == kProducer * 32) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&s.full[i], 1);
@@ -640,7 +632,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     int bkind = -1, bseg = -2;  // what B holds
     bool dep = false;           // grid dependency resolved for this thread
     bool flushed = false;       // gate/up count of this CTA published
-    bool dphase = false;
     float acc[2][4];
     int ru = 0;
     auto marker = [&](int m) {  // a hand-off without a tile: -1 end, -2 publish
@@ -655,16 +646,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         const int slot = gi % kStages;
         if (!mbar_wait(&s.full[slot], (gi / kStages) & 1)) { fail(a, s); return; }
         const int u = s.meta_u[slot], c = s.meta_c[slot];
-        if (u < 0 && threadIdx.x == 0) STMAX(11);
         if (u < 0) {  // end of work: publish (if still due) and tell the epilogue
             if ((!flushed && !marker(-2)) || !marker(-1)) fail(a, s);
             return;
         }
         const Unit un = unit_of<WF>(u, usg, u < usg ? 0 : s.n_seg, usd);
-        if ((un.kind == kDsh || un.kind == kDrt) && !dphase) { dphase = true; if (threadIdx.x == 0) { STMIN(8); STMAX(13); } }
         if (un.kind != kGsh && !dep) {
             grid_dep_wait();
-            if (threadIdx.x == 0) { STMIN(6); STMAX(9); }
             dep = true;
         }
         // B depends on the kind, and for down units on the expert (its h rows)
@@ -755,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 #pragma unroll
             for (int m = 0; m < 2; ++m)
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) sw[m][hh] = lds32(ss + 1024 * m + (g + 8 * hh) * 64 + 4 * warp);
+                for (int hh = 0; hh < 2; ++hh) sw[m][hh] = lds32(ss + 1024 * m + scale_off(g + 8 * hh, warp));
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc)
                 if (cc == c)
@@ -776,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) sw[t][hh] = lds32(ss + (16 * t + g + 8 * hh) * 64 + 4 * warp);
+                for (int hh = 0; hh < 2; ++hh) sw[t][hh] = lds32(ss + scale_off(16 * t + g + 8 * hh, warp));
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
@@ -817,7 +805,6 @@ __global__ void __launch_bounds__(256) decode_logits_kernel(const uint16_t *__re
                                                             float *__restrict__ logits, float2 *__restrict__ xscale) {
     __shared__ uint4 ws4[16 * 32];
     const int t = threadIdx.x >> 5, lane = threadIdx.x & 31, e = blockIdx.x;
-    if (threadIdx.x == 0) STMIN(0);
     constexpr int chunk = kD / 32;  // 128 elements = 16 uint4 per lane
     for (int i = threadIdx.x; i < 16 * 32; i += blockDim.x)
         cp_async_16(&ws4[i], wr + (int64_t)e * kD + (i & 31) * chunk + 8 * (i >> 5));
@@ -826,7 +813,6 @@ __global__ void __launch_bounds__(256) decode_logits_kernel(const uint16_t *__re
     for (int v = 0; v < 16; ++v) xv[v] = ldg128(x + (int64_t)t * kD + lane * chunk + 8 * v);
     cp_async_wait_all();
     __syncthreads();
-    if (threadIdx.x == 0) STMAX(1);
     grid_dep_launch();
     if (e == 0) {  // 2^p with max|x_t| 2^-p in [2^14, 2^15)
         float mx = 0.f;
@@ -859,7 +845,6 @@ __global__ void __launch_bounds__(256) decode_logits_kernel(const uint16_t *__re
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
     if (lane == 0) logits[(int64_t)t * E + e] = bias ? __fadd_rn(acc, bias[e]) : acc;
-    if (lane == 0) STMAX(3);
 }
 
 struct FinalizeArgs {
@@ -880,9 +865,7 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
     grid_dep_launch();
     for (int i = threadIdx.x; i < E + 2; i += blockDim.x) a.counters[i] = 0u;
     for (int i = threadIdx.x; i < T * k; i += blockDim.x) a.hmax[i] = 0u;
-    if (threadIdx.x == 0) STMIN(2);
     grid_dep_wait();
-    if (threadIdx.x == 0) STMAX(5);
     for (int base = 0; base < T * E; base += 8 * 256) {  // 8 loads in flight per thread
         float v[8];
 #pragma unroll
@@ -898,7 +881,6 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
     }
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = run[e] = 0;
     __syncthreads();
-    if (threadIdx.x == 0) STMAX(10);
     if (warp < T) {  // top-k + gates of token `warp`: lane holds experts lane + 32 i
         const float *l = lg + warp * E;
         float cv[32];
@@ -916,7 +898,6 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
         }
     }
     __syncthreads();
-    if (threadIdx.x == 0) STMAX(12);
     const int S = T * k;
     if (threadIdx.x < S) atomicAdd(&hist[sidx[threadIdx.x]], 1);
     __syncthreads();
@@ -941,7 +922,6 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
         if (lane == 31) a.offsets[E] = incl;
     }
     __syncthreads();
-    if (threadIdx.x == 0) STMAX(14);
     // stable rank of each slot among the earlier slots of its expert: within a
     // warp by matching lanes, across warps through a running count per expert
     for (int w0 = 0; w0 * 32 < S; ++w0) {
@@ -960,7 +940,6 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
         }
         __syncthreads();
     }
-    if (threadIdx.x == 0) STMAX(7);
 }
 
 // Stage-API entry (no routing in this call): the x prescale and the scratch reset.
@@ -1091,9 +1070,9 @@ cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uin
         ok = make_chunked_map(&a.m1c, p1 + L1.codes, r13, kD / 2, 16, 8) &&
              make_chunked_map(&a.m3c, p3 + L1.codes, r13, kD / 2, 16, 8) &&
              make_chunked_map(&a.m2c, p2 + L2.codes, r2, kF / 2, 32, 8) &&
-             make_plain_map(&a.m1s, p1 + L1.srow, r13, kD / 32, 64, 16) &&
-             make_plain_map(&a.m3s, p3 + L1.srow, r13, kD / 32, 64, 16) &&
-             make_plain_map(&a.m2s, p2 + L2.srow, r2, kF / 32, 64, 32);
+             make_plain_map(&a.m1s, p1 + L1.srow, r13, kD / 32, 64, 16, true) &&
+             make_plain_map(&a.m3s, p3 + L1.srow, r13, kD / 32, 64, 16, true) &&
+             make_plain_map(&a.m2s, p2 + L2.srow, r2, kF / 32, 64, 32, true);
     }
     if (ok && shared_out)
         ok = make_chunked_map(&a.ms1, w.sw1, d.d_ff_shared, kD * 2, 16, 8) &&

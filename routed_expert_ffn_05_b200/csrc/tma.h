@@ -17,10 +17,13 @@ namespace moe {
 bool make_chunked_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows,
                       uint32_t box_chunks);
 
-// A row-major byte matrix [rows][row_bytes] as 2D without swizzle, box
-// (box_bytes, box_rows). box_bytes a multiple of 16.
+// A row-major byte matrix [rows][row_bytes] as 2D, box (box_bytes, box_rows),
+// box_bytes a multiple of 16. swizzle64 (box_bytes == 64, shared-memory
+// destination 512-byte aligned): the 16-byte unit c of box row r lands at
+// unit c ^ ((r / 2) % 4), so one 4-byte word per row for 8 consecutive rows
+// falls in 8 different banks.
 bool make_plain_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_bytes,
-                    uint32_t box_rows);
+                    uint32_t box_rows, bool swizzle64 = false);
 
 // Operand tiles for the tensor-core GEMMs: a row-major matrix [rows][K]
 // seen in boxes of 128 K-elements x box_rows rows, 128-byte swizzled (rows of

@@ -28,6 +28,17 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(M, n) or n == "moe_status_string", n
 
 
+def test_library_exports_nothing_undeclared():
+    # the shared object's dynamic symbol table holds exactly the header's entry points
+    import subprocess
+    import routed_expert_ffn_05_b200 as M
+    out = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("nm unavailable")
+    exported = {l.split()[-1] for l in out.stdout.splitlines() if " T " in l}
+    assert exported == set(declared_functions()), sorted(exported ^ set(declared_functions()))
+
+
 def test_host_side_argument_checks():
     import routed_expert_ffn_05_b200 as M
     d = M.make_dims(4, 4096, 2048, 256, 8)
