@@ -186,14 +186,23 @@ __device__ __forceinline__ void arm(Smem &s, int slot, int u, int c, uint32_t tx
     mbar_arrive_expect_tx(&s.full[slot], tx);
 }
 
-// One 32-block of MXFP4 rows (r0 + g, r0 + g + 8 of a box with `rows` rows,
-// block = 16-byte unit `unit` of chunk `chunk`) against B.
-__device__ __forceinline__ void mxfp4_block(float acc[4], const uint8_t *box, int rows, int chunk, int unit, int r0,
-                                            int g, int q, uint32_t sw_lo, uint32_t sw_hi, int sj,
+// Shared-memory word loads at a 32-bit address plus a compile-time offset.
+template <int OFF>
+__device__ __forceinline__ uint32_t lds32_at(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
+    return v;
+}
+
+// One 32-block of MXFP4 rows against B: `addr` is lane (g, q)'s code word of
+// row g (16-byte unit of the block, swizzled, + 4 q); row g + 8 sits 1024
+// bytes (8 rows of 128) further. sl / sh: the rows' E8M0 scale words, byte sj.
+template <int OFF>
+__device__ __forceinline__ void mxfp4_block(float acc[4], uint32_t addr, uint32_t sw_lo, uint32_t sw_hi, int sj,
                                             const uint32_t b[4]) {
     uint32_t al[4], ah[4];
-    e2m1x8_to_f16x8(lds32(box + swz_off(chunk, rows, r0 + g, unit) + 4 * q), al);
-    e2m1x8_to_f16x8(lds32(box + swz_off(chunk, rows, r0 + g + 8, unit) + 4 * q), ah);
+    e2m1x8_to_f16x8(lds32_at<OFF>(addr), al);
+    e2m1x8_to_f16x8(lds32_at<OFF + 1024>(addr), ah);
     float t[4];
     mma_f16_16816_z(t, al[0], ah[0], al[1], ah[1], b[0], b[1]);
     mma_f16_16816(t, al[2], ah[2], al[3], ah[3], b[2], b[3]);
@@ -632,8 +641,19 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     int bkind = -1, bseg = -2;  // what B holds
     bool dep = false;           // grid dependency resolved for this thread
     bool flushed = false;       // gate/up count of this CTA published
+    int nseg = -1;              // active experts (read once, after routing)
     float acc[2][4];
     int ru = 0;
+    // Shared-memory addresses that stay fixed over stages. MXFP4 code words of
+    // this lane: block jj of the warp's K slice is 16-byte unit 4 (w & 1) + jj
+    // of chunk w / 2, rows g (+ 8 at +1024); a down box has 32 rows per chunk.
+    // The unit index is xor-swizzled with g, so its bits 4..5 vary with jj
+    // only through jj ^ (g & 3).
+    const uint32_t w_base = smem_u32(s.w[0]), s_base = smem_u32(s.s[0]);
+    const uint32_t code_gu = (uint32_t)swz_off(warp >> 1, 16, g, 4 * (warp & 1)) + 4 * q;
+    const uint32_t code_dn = (uint32_t)swz_off(warp >> 1, 32, g, 4 * (warp & 1)) + 4 * q;
+    const uint32_t sc_lo = (uint32_t)scale_off(g, warp), sc_hi = (uint32_t)scale_off(g + 8, warp);
+    auto code_off = [&](uint32_t base, int jj) { return base ^ ((uint32_t)jj << 4); };
     auto marker = [&](int m) {  // a hand-off without a tile: -1 end, -2 publish
         const int rb = ru & 1;
         if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) return false;
@@ -642,15 +662,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         ++ru;
         return true;
     };
-    for (int gi = 0;; ++gi) {
-        const int slot = gi % kStages;
-        if (!mbar_wait(&s.full[slot], (gi / kStages) & 1)) { fail(a, s); return; }
-        const int u = s.meta_u[slot], c = s.meta_c[slot];
+    auto release = [&](int slot) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[slot]);
+    };
+    int gi = 0;
+    auto next_stage = [&]() {  // the unit's next stage: wait until its data is in
+        ++gi;
+        return mbar_wait(&s.full[gi % kStages], (gi / kStages) & 1);
+    };
+    for (;; ++gi) {
+        if (!mbar_wait(&s.full[gi % kStages], (gi / kStages) & 1)) { fail(a, s); return; }
+        const int u = s.meta_u[gi % kStages];
         if (u < 0) {  // end of work: publish (if still due) and tell the epilogue
             if ((!flushed && !marker(-2)) || !marker(-1)) fail(a, s);
             return;
         }
-        const Unit un = unit_of<WF>(u, usg, u < usg ? 0 : s.n_seg, usd);
+        if (u >= usg && nseg < 0) nseg = s.n_seg;
+        const Unit un = unit_of<WF>(u, usg, u < usg ? 0 : nseg, usd);
         if (un.kind != kGsh && !dep) {
             grid_dep_wait();
             dep = true;
@@ -716,75 +745,91 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 }
             }
         }
-        if (c == 0 || un.kind == kDrt)
 #pragma unroll
-            for (int m = 0; m < 2; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
-        const uint8_t *st = s.w[slot], *ss = s.s[slot];
+        for (int m = 0; m < 2; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+        // The unit's stages, in order (the producer issues them back to back).
         if (un.kind == kGsh) {
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-                if (cc == c)
+            for (int c = 0; c < 8; ++c) {
+                if (c > 0 && !next_stage()) { fail(a, s); return; }
+                const uint8_t *st = s.w[gi % kStages];
 #pragma unroll
-                    for (int m = 0; m < 2; ++m) bf16_block(acc[m], st + 16384 * m, 16, warp, g, q, B[cc]);
+                for (int m = 0; m < 2; ++m) bf16_block(acc[m], st + 16384 * m, 16, warp, g, q, B[c]);
+                release(gi % kStages);
+            }
         } else if (Q2 && un.kind == kGrt) {
+            const int slot = gi % kStages;
+            const uint8_t *st = s.w[slot], *ss = s.s[slot];
 #pragma unroll
             for (int m = 0; m < 2; ++m)
                 q2k_superblock<-1>(acc[m], st + 16384 * m, ss + 4096 * m, ss + kQDd + 1024 * m, 16, 64, 0, warp, g,
                                    q, B, Bm);
+            release(slot);
         } else if (Q2 && un.kind == kDrt) {
+            const int slot = gi % kStages;
+            const uint8_t *st = s.w[slot], *ss = s.s[slot];
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 if (warp & 1) q2k_superblock<1>(acc[t], st, ss, ss + kQDd, 32, 32, 16 * t, warp >> 1, g, q, B, Bm);
                 else q2k_superblock<0>(acc[t], st, ss, ss + kQDd, 32, 32, 16 * t, warp >> 1, g, q, B, Bm);
             }
+            release(slot);
         } else if (un.kind == kGrt) {
-            // this warp's 4 blocks: 16-byte units 4 (w & 1) .. +3 of chunk w / 2; scale word w of each row
-            uint32_t sw[2][2];
+            // two stages of K 2048: W1 rows at +0, W3 rows at +16384; E8M0 scale
+            // word w of rows g, g + 8 (W3's 1024 bytes further)
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+            for (int c = 0; c < 2; ++c) {
+                if (c > 0 && !next_stage()) { fail(a, s); return; }
+                const int slot = gi % kStages;
+                const uint32_t cw = w_base + (uint32_t)slot * kStageW, cs = s_base + (uint32_t)slot * kStageS;
+                uint32_t sw[2][2];
+                sw[0][0] = lds32_at<0>(cs + sc_lo);
+                sw[0][1] = lds32_at<0>(cs + sc_hi);
+                sw[1][0] = lds32_at<1024>(cs + sc_lo);
+                sw[1][1] = lds32_at<1024>(cs + sc_hi);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) sw[m][hh] = lds32(ss + 1024 * m + scale_off(g + 8 * hh, warp));
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc)
-                if (cc == c)
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-                        for (int m = 0; m < 2; ++m)
-                            mxfp4_block(acc[m], st + 16384 * m, 16, warp >> 1, 4 * (warp & 1) + jj, 0, g, q, sw[m][0],
-                                        sw[m][1], jj, B[4 * cc + jj]);
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t ad = cw + code_off(code_gu, jj);
+                    mxfp4_block<0>(acc[0], ad, sw[0][0], sw[0][1], jj, B[4 * c + jj]);
+                    mxfp4_block<16384>(acc[1], ad, sw[1][0], sw[1][1], jj, B[4 * c + jj]);
+                }
+                release(slot);
+            }
         } else if (un.kind == kDsh) {
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc)
-                if (cc == c)
+            for (int c = 0; c < 2; ++c) {
+                if (c > 0 && !next_stage()) { fail(a, s); return; }
+                const uint8_t *st = s.w[gi % kStages];
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) bf16_block(acc[0], st, 16, 2 * warp + jj, g, q, B[2 * cc + jj]);
+                for (int jj = 0; jj < 2; ++jj) bf16_block(acc[0], st, 16, 2 * warp + jj, g, q, B[2 * c + jj]);
+                release(gi % kStages);
+            }
         } else {
+            // one stage: 32 W2 rows over all K; rows 16 t + g (+ 8)
+            const int slot = gi % kStages;
+            const uint32_t cw = w_base + (uint32_t)slot * kStageW, cs = s_base + (uint32_t)slot * kStageS;
             uint32_t sw[2][2];
+            sw[0][0] = lds32_at<0>(cs + sc_lo);
+            sw[0][1] = lds32_at<0>(cs + sc_hi);
+            sw[1][0] = lds32_at<1024>(cs + sc_lo);
+            sw[1][1] = lds32_at<1024>(cs + sc_hi);
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) sw[t][hh] = lds32(ss + scale_off(16 * t + g + 8 * hh, warp));
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-                for (int t = 0; t < 2; ++t)
-                    mxfp4_block(acc[t], st, 32, warp >> 1, 4 * (warp & 1) + jj, 16 * t, g, q, sw[t][0], sw[t][1], jj,
-                                B[jj]);
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint32_t ad = cw + code_off(code_dn, jj);
+                mxfp4_block<0>(acc[0], ad, sw[0][0], sw[0][1], jj, B[jj]);
+                mxfp4_block<2048>(acc[1], ad, sw[1][0], sw[1][1], jj, B[jj]);
+            }
+            release(slot);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.empty[slot]);
-        const bool last = un.kind == kDrt || c == un.nst - 1;
-        if (last) {  // hand the unit (or tile) to the epilogue warp
-            const int rb = ru & 1;
-            if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
-            const int rg = (un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;  // bf16 tiles read rows sigma(g)
-            put_partial(s.red[rb][warp][0], rg, q, acc[0]);
-            if (un.kind != kDsh) put_partial(s.red[rb][warp][1], rg, q, acc[1]);
-            if (threadIdx.x == 0) s.rmeta[rb] = u * 8 + c;
-            mbar_arrive(&s.rfull[rb]);
-            ++ru;
-        }
+        // hand the unit (or tile) to the epilogue warp
+        const int rb = ru & 1;
+        if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
+        const int rg = (un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;  // bf16 tiles read rows sigma(g)
+        put_partial(s.red[rb][warp][0], rg, q, acc[0]);
+        if (un.kind != kDsh) put_partial(s.red[rb][warp][1], rg, q, acc[1]);
+        if (threadIdx.x == 0) s.rmeta[rb] = u * 8 + (un.nst - 1);
+        mbar_arrive(&s.rfull[rb]);
+        ++ru;
     }
 }
 
