@@ -53,6 +53,11 @@ constexpr int kStageS = 10240;            // scale / metadata bytes per stage (M
                                           // Q2_K: 8 KB of sc|m bytes + 2 KB of (d, dmin))
 constexpr int kQDd = 8192;                // Q2_K: offset of the (d, dmin) pairs in a stage's metadata
 constexpr int kMaxE = 1024;
+// Partial tiles: element (matrix m, row r < 16, column c < 8) of a consumer
+// warp's 16x8 tiles at m * 144 + r * 9 + c. One column over all 16 rows and
+// both matrices then falls in 32 different banks (the epilogue reads by
+// column); the consumers' fragment stores conflict at most 2-way.
+constexpr int kRedM = 144, kRedR = 9, kRedW = 2 * kRedM;
 constexpr int kD = 4096, kF = 2048;       // the dims this tiling is written for
 constexpr int kGuTiles = kF / 16;         // gate/up tiles per routed expert
 constexpr int kDnTiles = kD / 32;         // down tiles (32 rows) per routed expert
@@ -84,7 +89,7 @@ struct DecodeArgs {
 struct Smem {
     uint8_t w[kStages][kStageW];
     uint8_t s[kStages][kStageS];
-    float red[2][kCW][2][128];   // partial 16x8 tiles per consumer warp
+    float red[2][kCW][kRedW];    // partial 16x8 tiles per consumer warp (see put_partial)
     uint64_t full[kStages], empty[kStages], rfull[2], rempty[2];
     int meta_u[kStages], meta_c[kStages];
     int rmeta[2];
@@ -224,13 +229,13 @@ __device__ __forceinline__ void bf16_block(float acc[4], const uint8_t *box, int
     mma_bf16_16816(acc, r0.z, r1.z, r0.w, r1.w, b[2], b[3]);
 }
 
-// C fragment -> partial tile [row][column]; MMA rows g, g + 8 land at rows
-// rg, rg + 8.
+// C fragment -> partial tile (rows r, columns c at r * 9 + c); MMA rows g,
+// g + 8 land at rows rg, rg + 8.
 __device__ __forceinline__ void put_partial(float *r, int rg, int q, const float acc[4]) {
-    r[rg * 8 + 2 * q] = acc[0];
-    r[rg * 8 + 2 * q + 1] = acc[1];
-    r[(rg + 8) * 8 + 2 * q] = acc[2];
-    r[(rg + 8) * 8 + 2 * q + 1] = acc[3];
+    r[rg * kRedR + 2 * q] = acc[0];
+    r[rg * kRedR + 2 * q + 1] = acc[1];
+    r[(rg + 8) * kRedR + 2 * q] = acc[2];
+    r[(rg + 8) * kRedR + 2 * q + 1] = acc[3];
 }
 
 // Byte offset of scale word w (the E8M0 bytes of 32-blocks 4w .. 4w + 3) of
@@ -550,49 +555,46 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 continue;
             }
             const Unit un = unit_of<WF>(m >> 3, usg, n, usd);
-            const float(*red)[2][128] = s.red[rb];
-            // Partial tiles are [row][column] per consumer warp; each lane sums
-            // 4 columns of one row across the warps with 16-byte loads.
-            auto sum4 = [&](int mat, int off) {
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            // Sum over the consumer warps of one column: lane l takes matrix
+            // (or down row half) l / 16, row l % 16 (four chains for latency).
+            const float *red = &s.red[rb][0][0] + (lane >> 4) * kRedM + (lane & 15) * kRedR;
+            auto colsum = [&](int c) {
+                float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
 #pragma unroll
-                for (int w = 0; w < kCW; ++w) {
-                    const float4 p = *reinterpret_cast<const float4 *>(&red[w][mat][off]);
-                    v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+                for (int w = 0; w < kCW; w += 4) {
+                    v0 += red[w * kRedW + c];
+                    v1 += red[(w + 1) * kRedW + c];
+                    v2 += red[(w + 2) * kRedW + c];
+                    v3 += red[(w + 3) * kRedW + c];
                 }
-                return v;
+                return (v0 + v1) + (v2 + v3);
             };
-            auto pick = [](const float4 &v, int c) { return c == 0 ? v.x : (c == 1 ? v.y : (c == 2 ? v.z : v.w)); };
+            const int row = lane & 15;
             if (un.kind == kGsh || un.kind == kGrt) {
-                // lane: row l / 2 of the 16-row tile, columns 4 (l % 2) .. +3
-                const int row = lane >> 1, half = lane & 1, col = 16 * un.tile + row;
-                const float4 g4 = sum4(0, row * 8 + 4 * half), u4 = sum4(1, row * 8 + 4 * half);
+                // lanes 0..15: gate of rows 0..15, lanes 16..31: up
+                const int col = 16 * un.tile + row;
                 if (un.kind == kGsh) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int tok = 4 * half + c;
-                        if (tok < a.T)
-                            a.hs[(int64_t)tok * a.Fs + col] =
-                                f32_to_bf16_rne(silu_f32(pick(g4, c)) * pick(u4, c));
+                    for (int c = 0; c < a.T; ++c) {
+                        const float v = colsum(c);
+                        const float up = __shfl_down_sync(0xffffffffu, v, 16);
+                        if (lane < 16) a.hs[(int64_t)c * a.Fs + col] = f32_to_bf16_rne(silu_f32(v) * up);
                     }
+                    ++sh_fin;
                 } else {
                     const int rbase = s.ep_rbase[un.seg], cnt = s.ep_cnt[un.seg];
                     for (int i = 0; i < cnt; ++i) {  // the expert's rows; column = the row's token
                         const int tok = s.ep_tok[un.seg][i];
-                        const bool mine = (tok >> 2) == half;
+                        const float xs = s.ep_xs[tok];
+                        const float v = colsum(tok);
+                        const float up = __shfl_down_sync(0xffffffffu, v, 16);
                         uint32_t hb = 0;
-                        if (mine) {
-                            const float xs = s.ep_xs[tok];
-                            hb = f32_to_bf16_rne(silu_f32(pick(g4, tok & 3) * xs) * (pick(u4, tok & 3) * xs));
+                        if (lane < 16) {
+                            hb = f32_to_bf16_rne(silu_f32(v * xs) * (up * xs));
                             a.h[(int64_t)(rbase + i) * kF + col] = (uint16_t)hb;
                         }
                         const uint32_t mx = warp_max_bits((hb & 0x7FFFu) << 16);
                         if (lane == 0) atomicMax(&a.hmax[rbase + i], mx);
                     }
-                }
-                if (un.kind == kGsh) {
-                    ++sh_fin;
-                } else {
                     if (un.seg != pseg) {  // a new expert: the previous one's count goes out
                         publish();
                         pseg = un.seg;
@@ -600,12 +602,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     ++r_fin;
                 }
             } else if (un.kind == kDsh) {
-                const int row = lane >> 1, half = lane & 1;
-                const float4 v4 = sum4(0, row * 8 + 4 * half);
+                // one matrix: lanes 0..15 and 16..31 take alternate columns
+                for (int c = lane >> 4; c < a.T; c += 2) {
+                    const float *r0 = &s.red[rb][0][0] + row * kRedR + c;
+                    float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int tok = 4 * half + c;
-                    if (tok < a.T) a.shared_out[(int64_t)tok * kD + 16 * un.tile + row] = pick(v4, c);
+                    for (int w = 0; w < kCW; w += 2) {
+                        v0 += r0[w * kRedW];
+                        v1 += r0[(w + 1) * kRedW];
+                    }
+                    a.shared_out[(int64_t)c * kD + 16 * un.tile + row] = v0 + v1;
                 }
             } else {
                 // lane = row of the 32-row tile; columns = the expert's rows
@@ -614,14 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     dseg = un.seg;
                     dsc = lane < cnt ? row_scale(__ldcg(&a.hmax[rbase + lane])) : 1.f;
                 }
-                const int t = lane >> 4, r16 = lane & 15;
-                const float4 lo = sum4(t, r16 * 8), hi = sum4(t, r16 * 8 + 4);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < cnt; ++i) {
                     const float sc = __shfl_sync(0xffffffffu, dsc, i);
-                    if (i < cnt)
-                        a.out_rows[(int64_t)(rbase + i) * kD + 32 * un.tile + lane] =
-                            (i < 4 ? pick(lo, i) : pick(hi, i - 4)) * sc;
+                    a.out_rows[(int64_t)(rbase + i) * kD + 32 * un.tile + lane] = colsum(i) * sc;
                 }
             }
             __syncwarp();
@@ -825,8 +826,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         const int rb = ru & 1;
         if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
         const int rg = (un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;  // bf16 tiles read rows sigma(g)
-        put_partial(s.red[rb][warp][0], rg, q, acc[0]);
-        if (un.kind != kDsh) put_partial(s.red[rb][warp][1], rg, q, acc[1]);
+        put_partial(s.red[rb][warp], rg, q, acc[0]);
+        if (un.kind != kDsh) put_partial(s.red[rb][warp] + kRedM, rg, q, acc[1]);
         if (threadIdx.x == 0) s.rmeta[rb] = u * 8 + (un.nst - 1);
         mbar_arrive(&s.rfull[rb]);
         ++ru;
