@@ -47,10 +47,14 @@ constexpr int kCW = 16;                   // consumer warps (each owns 1/16 of K
 constexpr int kProducer = kCW;            // warp index of the producer
 constexpr int kEpilogue = kCW + 1;        // warp index of the epilogue warp
 constexpr int kThreads = (kCW + 2) * 32;
-constexpr int kStages = 4;
 constexpr int kStageW = 32768;            // weight tile bytes per stage
-constexpr int kStageS = 10240;            // scale / metadata bytes per stage (MXFP4: 2 KB of E8M0;
-                                          // Q2_K: 8 KB of sc|m bytes + 2 KB of (d, dmin))
+// Stages and per-stage scale / metadata bytes by weight format: MXFP4 needs
+// 2 KB of E8M0 per stage, so five stages fit; Q2_K needs 8 KB of sc|m bytes
+// and 2 KB of (d, dmin) and keeps four.
+template <int WF> struct Pipe {
+    static constexpr int stages = WF == MOE_W_Q2K ? 4 : 5;
+    static constexpr int meta = WF == MOE_W_Q2K ? 10240 : 2048;
+};
 constexpr int kQDd = 8192;                // Q2_K: offset of the (d, dmin) pairs in a stage's metadata
 constexpr int kMaxE = 1024;
 // Partial tiles: element (matrix m, row r < 16, column c < 8) of a consumer
@@ -86,9 +90,11 @@ struct DecodeArgs {
     int *err;
 };
 
+template <int WF>
 struct Smem {
+    static constexpr int kStages = Pipe<WF>::stages;
     uint8_t w[kStages][kStageW];
-    uint8_t s[kStages][kStageS];
+    uint8_t s[kStages][Pipe<WF>::meta];
     float red[2][kCW][kRedW];    // partial 16x8 tiles per consumer warp (see put_partial)
     uint64_t full[kStages], empty[kStages], rfull[2], rempty[2];
     int meta_u[kStages], meta_c[kStages];
@@ -103,10 +109,13 @@ struct Smem {
     uint8_t ep_tok[kMaxE][8];
     float ep_xs[8];
 };
-constexpr int kSmemBytes = (int)sizeof(Smem) + 1024;  // + alignment slack
+template <int WF> constexpr int smem_bytes() { return (int)sizeof(Smem<WF>) + 1024; }  // + alignment slack
+static_assert(smem_bytes<MOE_W_MXFP4>() <= 227 * 1024 && smem_bytes<MOE_W_Q2K>() <= 227 * 1024,
+              "decode kernel shared memory");
 
-__device__ __forceinline__ Smem &smem_ref(uint8_t *raw) {
-    return *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+template <int WF>
+__device__ __forceinline__ Smem<WF> &smem_ref(uint8_t *raw) {
+    return *reinterpret_cast<Smem<WF> *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
 }
 
 __device__ __forceinline__ uint4 ldg128(const void *p) { return __ldg(reinterpret_cast<const uint4 *>(p)); }
@@ -164,7 +173,8 @@ __device__ __forceinline__ Unit unit_of(int u, int usg, int n_seg, int usd) {
     return Unit{kDrt, r / kDnTiles, r % kDnTiles, 1};
 }
 
-__device__ __forceinline__ void fail(const DecodeArgs &a, Smem &s) {
+template <class S>
+__device__ __forceinline__ void fail(const DecodeArgs &a, S &s) {
     set_device_error(a.err, MOE_DEVERR_TIMEOUT);
     s.abort = 1;
 }
@@ -185,7 +195,8 @@ __device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t target, i
     return ok;
 }
 
-__device__ __forceinline__ void arm(Smem &s, int slot, int u, int c, uint32_t tx) {
+template <class S>
+__device__ __forceinline__ void arm(S &s, int slot, int u, int c, uint32_t tx) {
     s.meta_u[slot] = u;
     s.meta_c[slot] = c;
     mbar_arrive_expect_tx(&s.full[slot], tx);
@@ -379,8 +390,9 @@ __device__ __forceinline__ void q2k_load_b(const uint16_t *row, float inv, int q
 template <int WF>
 __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr bool Q2 = WF == MOE_W_Q2K;
+    constexpr int kStages = Pipe<WF>::stages, kStageS = Pipe<WF>::meta;
     extern __shared__ uint8_t smem_raw[];
-    Smem &s = smem_ref(smem_raw);
+    Smem<WF> &s = smem_ref<WF>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == kProducer * 32) {
         for (int i = 0; i < kStages; ++i) {
@@ -388,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             mbar_init(&s.empty[i], kCW);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.rfull[i], kCW * 32);
+            mbar_init(&s.rfull[i], kCW);  // one arrival per consumer warp
             mbar_init(&s.rempty[i], 1);
         }
         s.abort = 0;
@@ -650,16 +662,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     // of chunk w / 2, rows g (+ 8 at +1024); a down box has 32 rows per chunk.
     // The unit index is xor-swizzled with g, so its bits 4..5 vary with jj
     // only through jj ^ (g & 3).
-    const uint32_t w_base = smem_u32(s.w[0]), s_base = smem_u32(s.s[0]);
+    // (A down box's chunks hold 32 rows: its code word sits 2048 (w / 2) bytes
+    // further than a gate/up box's. Scale rows g + 8 sit 512 bytes after row g:
+    // the swizzle term depends on (row / 2) % 4 only.)
+    const uint32_t w_base = smem_u32(s.w[0]);
+    constexpr uint32_t kScaleBase = (uint32_t)(kStages * kStageW);  // s.s[0] - s.w[0]
     const uint32_t code_gu = (uint32_t)swz_off(warp >> 1, 16, g, 4 * (warp & 1)) + 4 * q;
-    const uint32_t code_dn = (uint32_t)swz_off(warp >> 1, 32, g, 4 * (warp & 1)) + 4 * q;
-    const uint32_t sc_lo = (uint32_t)scale_off(g, warp), sc_hi = (uint32_t)scale_off(g + 8, warp);
+    const uint32_t sc_lo = (uint32_t)scale_off(g, warp);
     auto code_off = [&](uint32_t base, int jj) { return base ^ ((uint32_t)jj << 4); };
     auto marker = [&](int m) {  // a hand-off without a tile: -1 end, -2 publish
         const int rb = ru & 1;
         if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) return false;
         if (threadIdx.x == 0) s.rmeta[rb] = m;
-        mbar_arrive(&s.rfull[rb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.rfull[rb]);
         ++ru;
         return true;
     };
@@ -782,12 +798,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             for (int c = 0; c < 2; ++c) {
                 if (c > 0 && !next_stage()) { fail(a, s); return; }
                 const int slot = gi % kStages;
-                const uint32_t cw = w_base + (uint32_t)slot * kStageW, cs = s_base + (uint32_t)slot * kStageS;
+                const uint32_t cw = w_base + (uint32_t)slot * kStageW;
+                const uint32_t cs = w_base + kScaleBase + (uint32_t)slot * kStageS + sc_lo;
                 uint32_t sw[2][2];
-                sw[0][0] = lds32_at<0>(cs + sc_lo);
-                sw[0][1] = lds32_at<0>(cs + sc_hi);
-                sw[1][0] = lds32_at<1024>(cs + sc_lo);
-                sw[1][1] = lds32_at<1024>(cs + sc_hi);
+                sw[0][0] = lds32_at<0>(cs);
+                sw[0][1] = lds32_at<512>(cs);
+                sw[1][0] = lds32_at<1024>(cs);
+                sw[1][1] = lds32_at<1536>(cs);
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                     const uint32_t ad = cw + code_off(code_gu, jj);
@@ -808,15 +825,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         } else {
             // one stage: 32 W2 rows over all K; rows 16 t + g (+ 8)
             const int slot = gi % kStages;
-            const uint32_t cw = w_base + (uint32_t)slot * kStageW, cs = s_base + (uint32_t)slot * kStageS;
+            const uint32_t cw = w_base + (uint32_t)slot * kStageW + 2048u * (uint32_t)(warp >> 1);
+            const uint32_t cs = w_base + kScaleBase + (uint32_t)slot * kStageS + sc_lo;
             uint32_t sw[2][2];
-            sw[0][0] = lds32_at<0>(cs + sc_lo);
-            sw[0][1] = lds32_at<0>(cs + sc_hi);
-            sw[1][0] = lds32_at<1024>(cs + sc_lo);
-            sw[1][1] = lds32_at<1024>(cs + sc_hi);
+            sw[0][0] = lds32_at<0>(cs);
+            sw[0][1] = lds32_at<512>(cs);
+            sw[1][0] = lds32_at<1024>(cs);
+            sw[1][1] = lds32_at<1536>(cs);
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t ad = cw + code_off(code_dn, jj);
+                const uint32_t ad = cw + code_off(code_gu, jj);
                 mxfp4_block<0>(acc[0], ad, sw[0][0], sw[0][1], jj, B[jj]);
                 mxfp4_block<2048>(acc[1], ad, sw[1][0], sw[1][1], jj, B[jj]);
             }
@@ -829,7 +847,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         put_partial(s.red[rb][warp], rg, q, acc[0]);
         if (un.kind != kDsh) put_partial(s.red[rb][warp] + kRedM, rg, q, acc[1]);
         if (threadIdx.x == 0) s.rmeta[rb] = u * 8 + (un.nst - 1);
-        mbar_arrive(&s.rfull[rb]);
+        __syncwarp();  // the warp's tile stores, then one arrival (release) for the warp
+        if (lane == 0) mbar_arrive(&s.rfull[rb]);
         ++ru;
     }
 }
@@ -1025,10 +1044,10 @@ cudaError_t set_smem_attrs() {
     if (done[dev]) return cudaSuccess;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(decode_ffn_kernel<MOE_W_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  kSmemBytes)))
+                                  smem_bytes<MOE_W_MXFP4>())))
         return e;
     if ((e = cudaFuncSetAttribute(decode_ffn_kernel<MOE_W_Q2K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  kSmemBytes)))
+                                  smem_bytes<MOE_W_Q2K>())))
         return e;
     done[dev] = true;
     return cudaSuccess;
@@ -1141,8 +1160,9 @@ cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uin
                                               a.counters);
         count_launches(1);
     }
-    e = q2 ? launch_pdl(decode_ffn_kernel<MOE_W_Q2K>, dim3(num_sms()), dim3(kThreads), kSmemBytes, s, a)
-           : launch_pdl(decode_ffn_kernel<MOE_W_MXFP4>, dim3(num_sms()), dim3(kThreads), kSmemBytes, s, a);
+    e = q2 ? launch_pdl(decode_ffn_kernel<MOE_W_Q2K>, dim3(num_sms()), dim3(kThreads), smem_bytes<MOE_W_Q2K>(), s, a)
+           : launch_pdl(decode_ffn_kernel<MOE_W_MXFP4>, dim3(num_sms()), dim3(kThreads), smem_bytes<MOE_W_MXFP4>(), s,
+                        a);
     if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
