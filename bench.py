@@ -321,7 +321,7 @@ def oracle_sample(cfg, T, n_tokens, min_seconds, seed=0, batch=0):
         oracle.layer_tokens(ow, x, toks, tok)
         reps += 1
         el = time.perf_counter() - t0
-        if el >= min_seconds or reps >= 20:
+        if el >= min_seconds or reps >= 200:
             break
     return reps * n_tokens / el, oracle.num_threads(), el, \
         f"{reps} x oracle layer on {n_tokens} token(s) of the {cfg.name} T={T} batch"
