@@ -97,7 +97,7 @@ struct Smem {
     uint8_t s[kStages][Pipe<WF>::meta];
     float red[2][kCW][kRedW];    // partial 16x8 tiles per consumer warp (see put_partial)
     uint64_t full[kStages], empty[kStages], rfull[2], rempty[2];
-    int meta_u[kStages], meta_c[kStages];
+    int meta_u[kStages], meta_k[kStages];  // unit of the stage, and the unit decoded (pack_unit)
     int rmeta[2];
     int seg_e[kMaxE];
     int n_seg;
@@ -195,10 +195,17 @@ __device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t target, i
     return ok;
 }
 
+// A unit's fields in one word for the consumers: kind (2 bits), stages (4),
+// tile (8), active-expert segment (11; 0 for the shared expert).
+__device__ __forceinline__ int pack_unit(const Unit &un) {
+    return un.kind | un.nst << 2 | un.tile << 6 | max(un.seg, 0) << 14;
+}
+__device__ __forceinline__ Unit unpack_unit(int p) { return Unit{p & 3, p >> 14, (p >> 6) & 255, (p >> 2) & 15}; }
+
 template <class S>
-__device__ __forceinline__ void arm(S &s, int slot, int u, int c, uint32_t tx) {
+__device__ __forceinline__ void arm(S &s, int slot, int u, const Unit &un, uint32_t tx) {
     s.meta_u[slot] = u;
-    s.meta_c[slot] = c;
+    s.meta_k[slot] = pack_unit(un);
     mbar_arrive_expect_tx(&s.full[slot], tx);
 }
 
@@ -425,44 +432,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 const int slot = gi % kStages;
                 if (!mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1)) { fail(a, s); return; }
                 uint8_t *w = s.w[slot];
+                uint8_t *sm = &s.s[0][0] + (size_t)slot * kStageS;  // the stage's scale / metadata bytes
                 uint64_t *bar = &s.full[slot];
                 switch (un.kind) {
                     case kGsh:
-                        arm(s, slot, u, c, 2 * 16384);
+                        arm(s, slot, u, un, 2 * 16384);
                         tma_load_3d(w, &a.ms1, 0, 16 * un.tile, 8 * c, bar);
                         tma_load_3d(w + 16384, &a.ms3, 0, 16 * un.tile, 8 * c, bar);
                         break;
                     case kGrt:
                         if (Q2) {  // quants, sc|m bytes and (d, dmin) of 16 rows over all K
-                            arm(s, slot, u, c, 2 * 16384 + 2 * 4096 + 2 * 1024);
+                            arm(s, slot, u, un, 2 * 16384 + 2 * 4096 + 2 * 1024);
                             tma_load_3d(w, &a.m1c, 0, row0, 0, bar);
                             tma_load_3d(w + 16384, &a.m3c, 0, row0, 0, bar);
-                            tma_load_3d(s.s[slot], &a.m1s, 0, row0, 0, bar);
-                            tma_load_3d(s.s[slot] + 4096, &a.m3s, 0, row0, 0, bar);
-                            tma_load_2d(s.s[slot] + kQDd, &a.m1d, 0, row0, bar);
-                            tma_load_2d(s.s[slot] + kQDd + 1024, &a.m3d, 0, row0, bar);
+                            tma_load_3d(sm, &a.m1s, 0, row0, 0, bar);
+                            tma_load_3d(sm + 4096, &a.m3s, 0, row0, 0, bar);
+                            tma_load_2d(sm + kQDd, &a.m1d, 0, row0, bar);
+                            tma_load_2d(sm + kQDd + 1024, &a.m3d, 0, row0, bar);
                         } else {
-                            arm(s, slot, u, c, 2 * 16384 + 2 * 1024);
+                            arm(s, slot, u, un, 2 * 16384 + 2 * 1024);
                             tma_load_3d(w, &a.m1c, 0, row0, 8 * c, bar);
                             tma_load_3d(w + 16384, &a.m3c, 0, row0, 8 * c, bar);
-                            tma_load_2d(s.s[slot], &a.m1s, 64 * c, row0, bar);
-                            tma_load_2d(s.s[slot] + 1024, &a.m3s, 64 * c, row0, bar);
+                            tma_load_2d(sm, &a.m1s, 64 * c, row0, bar);
+                            tma_load_2d(sm + 1024, &a.m3s, 64 * c, row0, bar);
                         }
                         break;
                     case kDsh:
-                        arm(s, slot, u, c, 32768);
+                        arm(s, slot, u, un, 32768);
                         tma_load_3d(w, &a.ms2, 0, 16 * un.tile, 16 * c, bar);
                         break;
                     default:
                         if (Q2) {  // 32 rows of W2 over all K
-                            arm(s, slot, u, c, 16384 + 4096 + 1024);
+                            arm(s, slot, u, un, 16384 + 4096 + 1024);
                             tma_load_3d(w, &a.m2c, 0, row0, 0, bar);
-                            tma_load_3d(s.s[slot], &a.m2s, 0, row0, 0, bar);
-                            tma_load_2d(s.s[slot] + kQDd, &a.m2d, 0, row0, bar);
+                            tma_load_3d(sm, &a.m2s, 0, row0, 0, bar);
+                            tma_load_2d(sm + kQDd, &a.m2d, 0, row0, bar);
                         } else {
-                            arm(s, slot, u, c, 32768 + 2048);
+                            arm(s, slot, u, un, 32768 + 2048);
                             tma_load_3d(w, &a.m2c, 0, row0, 0, bar);
-                            tma_load_2d(s.s[slot], &a.m2s, 0, row0, bar);
+                            tma_load_2d(sm, &a.m2s, 0, row0, bar);
                         }
                 }
             }
@@ -654,7 +662,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     int bkind = -1, bseg = -2;  // what B holds
     bool dep = false;           // grid dependency resolved for this thread
     bool flushed = false;       // gate/up count of this CTA published
-    int nseg = -1;              // active experts (read once, after routing)
     float acc[2][4];
     int ru = 0;
     // Shared-memory addresses that stay fixed over stages. MXFP4 code words of
@@ -683,20 +690,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.empty[slot]);
     };
-    int gi = 0;
-    auto next_stage = [&]() {  // the unit's next stage: wait until its data is in
-        ++gi;
-        return mbar_wait(&s.full[gi % kStages], (gi / kStages) & 1);
+    int slot = 0;      // ring slot of the current stage
+    uint32_t ph = 0;   // its full-barrier parity
+    auto advance = [&]() {
+        if (++slot == kStages) {
+            slot = 0;
+            ph ^= 1u;
+        }
     };
-    for (;; ++gi) {
-        if (!mbar_wait(&s.full[gi % kStages], (gi / kStages) & 1)) { fail(a, s); return; }
-        const int u = s.meta_u[gi % kStages];
+    auto next_stage = [&]() {  // the unit's next stage: wait until its data is in
+        advance();
+        return mbar_wait(&s.full[slot], ph);
+    };
+    for (;; advance()) {
+        if (!mbar_wait(&s.full[slot], ph)) { fail(a, s); return; }
+        const int u = s.meta_u[slot];
         if (u < 0) {  // end of work: publish (if still due) and tell the epilogue
             if ((!flushed && !marker(-2)) || !marker(-1)) fail(a, s);
             return;
         }
-        if (u >= usg && nseg < 0) nseg = s.n_seg;
-        const Unit un = unit_of<WF>(u, usg, u < usg ? 0 : nseg, usd);
+        const Unit un = unpack_unit(s.meta_k[slot]);
         if (un.kind != kGsh && !dep) {
             grid_dep_wait();
             dep = true;
@@ -769,13 +782,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 if (c > 0 && !next_stage()) { fail(a, s); return; }
-                const uint8_t *st = s.w[gi % kStages];
+                const uint8_t *st = s.w[slot];
 #pragma unroll
                 for (int m = 0; m < 2; ++m) bf16_block(acc[m], st + 16384 * m, 16, warp, g, q, B[c]);
-                release(gi % kStages);
+                release(slot);
             }
         } else if (Q2 && un.kind == kGrt) {
-            const int slot = gi % kStages;
             const uint8_t *st = s.w[slot], *ss = s.s[slot];
 #pragma unroll
             for (int m = 0; m < 2; ++m)
@@ -783,7 +795,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                                    q, B, Bm);
             release(slot);
         } else if (Q2 && un.kind == kDrt) {
-            const int slot = gi % kStages;
             const uint8_t *st = s.w[slot], *ss = s.s[slot];
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
@@ -797,7 +808,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 if (c > 0 && !next_stage()) { fail(a, s); return; }
-                const int slot = gi % kStages;
                 const uint32_t cw = w_base + (uint32_t)slot * kStageW;
                 const uint32_t cs = w_base + kScaleBase + (uint32_t)slot * kStageS + sc_lo;
                 uint32_t sw[2][2];
@@ -817,14 +827,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 if (c > 0 && !next_stage()) { fail(a, s); return; }
-                const uint8_t *st = s.w[gi % kStages];
+                const uint8_t *st = s.w[slot];
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj) bf16_block(acc[0], st, 16, 2 * warp + jj, g, q, B[2 * c + jj]);
-                release(gi % kStages);
+                release(slot);
             }
         } else {
             // one stage: 32 W2 rows over all K; rows 16 t + g (+ 8)
-            const int slot = gi % kStages;
             const uint32_t cw = w_base + (uint32_t)slot * kStageW + 2048u * (uint32_t)(warp >> 1);
             const uint32_t cs = w_base + kScaleBase + (uint32_t)slot * kStageS + sc_lo;
             uint32_t sw[2][2];
