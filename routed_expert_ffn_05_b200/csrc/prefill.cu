@@ -7,19 +7,19 @@
 // hysenlabs.com, "Model support and quantisation"). The layer's math:
 // g = W1 a, u = W3 a, h = silu(g) * u quantised to MXFP8 along F, o = W2 h.
 //
-// Mapping onto tcgen05.mma (M = 128, K = 32 per instruction):
-//  - the MMA's M side is 128 weight rows and its N side is a tile of up to
-//    128 of the expert's tokens, trimmed to a multiple of 16. Routing is
-//    skewed (a Zipf-like expert popularity leaves many experts with a few
-//    tokens), so putting tokens on N costs at most 15 padded columns per tile
-//    where 128-row token tiles on M would cost up to 127 rows;
-//  - gate/up: two MMAs per K step (W1 and W3 tiles against the same token
-//    tile) into two 128-column fp32 accumulators, so SwiGLU pairs g and u in
-//    the same thread after tcgen05.ld; the h block amax along F (across the
-//    warp's 32 lanes = 32 consecutive weight rows) is one redux.sync;
-//  - down: two MMAs per K step as well, rows 256 f .. +127 and +128 .. +255
-//    of W2 against the same token tile, so each token tile is read once per
-//    256 output features (half the shared-memory and L2 traffic of 128);
+// Mapping onto tcgen05.mma (K = 32 per instruction):
+//  - A is a tile of 128 of the expert's tokens (M = 128, E4M3) and B is 256
+//    weight rows (N = 256, E2M1): for gate/up the 128 rows of W1 and the same
+//    128 rows of W3 stacked, for down 256 rows of W2. One MMA per K step then
+//    gives g and u (or 256 output features) for every token of the tile. An
+//    instruction costs the same at N = 128 as at N = 64 or 32 (its 128 x 32
+//    A read sets the time), and N = 256 costs ~1.1x N = 128, so one 256-wide
+//    MMA does the work of two 128-wide ones in ~55% of their time;
+//    token tiles that are not full (the routing is skewed, many experts get a
+//    few tokens) cost a full tile either way;
+//  - the epilogue thread is a token (a TMEM lane): SwiGLU pairs columns c and
+//    128 + c, the MXFP8 amax of h along F is 32 values of the same thread, and
+//    h codes and output rows leave as contiguous 16-byte stores;
 //  - operands arrive by TMA in 128-byte-swizzled K-major boxes of 128 K; E2M1
 //    codes are expanded to one byte per element in shared memory by the
 //    tensor map's 16U4_ALIGN16B type; the E8M0 scales come in 512-byte atoms
@@ -117,10 +117,9 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
     return r;
 }
 
-__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
-    uint32_t r;
-    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
-    return r;
+// Two fp32 -> bf16 (round to nearest even), the first in the low half.
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+    return (uint32_t)f32_to_bf16_rne(lo) | (uint32_t)f32_to_bf16_rne(hi) << 16;
 }
 
 // 2^-se as an fp32 (exact for se in [-127, 126]).
@@ -196,9 +195,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         if (lane == 0) {
             int it = 0, lw = 0;
             for (int w = blockIdx.x; w < n_work && !s.abort; w += gridDim.x, ++lw) {
-                const Work wk = work_of(w, ft, s.ustart, a.E, a.offsets);
-                const int n16 = (wk.nvalid + 15) & ~15;
-                const uint32_t idesc = idesc_mx(5, 0, 128, n16);
+                // A = the token tile (E4M3, M = 128), B = both 128-row weight tiles
+                // as one 256-row operand (E2M1, N = 256): one MMA per K step
+                // yields gate and up (or 256 down features) for every token
+                constexpr uint32_t idesc = idesc_mx(0, 5, 128, 256);
                 if (!mbar_wait(&s.acc_empty, (lw & 1) ^ 1)) { tc_fail(a, s); break; }
                 tc_fence_after();
                 bool ok = true;
@@ -206,18 +206,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                     const int slot = it % kTcStages;
                     if (!mbar_wait(&s.full[slot], (it / kTcStages) & 1)) { ok = false; break; }
                     tc_fence_after();
+                    // scale columns: weight rows 0..127 at +0, 128..255 at +4 (B reads
+                    // column n / 32), tokens at +8 (A reads column m / 32)
                     const uint32_t sfc = tmem + kSfCol + 16 * slot;
                     tc_cp_sf(sfc, sdesc_sf(s.sf[slot][0]));
                     tc_cp_sf(sfc + 4, sdesc_sf(s.sf[slot][1]));
                     tc_cp_sf(sfc + 8, sdesc_sf(s.sf[slot][2]));
-                    const uint64_t d0 = sdesc_sw128(s.a[slot][0]), d1 = sdesc_sw128(s.a[slot][1]),
-                                   db = sdesc_sw128(s.b[slot]);
+                    const uint64_t dt = sdesc_sw128(s.b[slot]), dw = sdesc_sw128(s.a[slot][0]);  // a[slot][0..1]: 256 rows
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint32_t id = idesc_sf_ids(idesc, ks, ks), acc = (kt | ks) != 0;
                         const uint32_t sel = (uint32_t)ks << 30;
-                        tc_mma_mx(tmem, d0 + 2 * ks, db + 2 * ks, id, sfc | sel, (sfc + 8) | sel, acc);
-                        tc_mma_mx(tmem + 128, d1 + 2 * ks, db + 2 * ks, id, (sfc + 4) | sel, (sfc + 8) | sel, acc);
+                        tc_mma_mx(tmem, dt + 2 * ks, dw + 2 * ks, id, (sfc + 8) | sel, sfc | sel, acc);
                     }
                     tc_commit(&s.empty[slot]);  // frees the stage once these MMAs finish
                 }
@@ -229,9 +229,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         }
     } else {
         // ------------------------------ epilogue ------------------------------
+        // TMEM lane = token of the tile (this warp: tokens 32 q .. 32 q + 31),
+        // column = weight row: gate/up g at 0..127 and u at 128..255, down the
+        // tile's 256 output features. Warp half h takes F rows 64 h .. +63
+        // (gate/up) or features 128 h .. +127 (down).
         const int q = warp & 3;              // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;    // token columns [64 half, 64 half + 64)
+        const int half = (warp - 2) >> 2;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        const int t = 32 * q + lane;         // this thread's token in the tile
         int lw = 0;
         // control flow stays warp-uniform: tcgen05.ld is a warp-collective
         for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++lw) {
@@ -243,91 +248,82 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                 break;
             }
             tc_fence_after();
+            const bool busy = 32 * q < wk.nvalid;  // warp-uniform: any valid token in this quarter
+            const bool valid = t < wk.nvalid;
             // Pull this warp's columns out of TMEM (gate/up: h = silu(g) u right
             // away), then hand the accumulator back before the slow part, so the
             // next tile's MMAs overlap the requantisation and the stores.
-            const int c0 = 64 * half;
-            const int nc = max(0, min(64, wk.nvalid - c0));  // this warp's valid columns
-            float v[64], v2[GU ? 1 : 64];  // down: v2 = the second 128 rows
-            if (nc > 0) {
+            float v[GU ? 64 : 128];
+            if (busy) {
                 uint32_t r[32];
+                if (GU) {
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    if (c * 32 < nc) {  // warp-uniform
-                        tmem_ld32(lane_base + c0 + 32 * c, r);
-                        if (GU) {
-                            uint32_t u[32];
-                            tmem_ld32(lane_base + 128 + c0 + 32 * c, u);
-                            tmem_wait_ld();
+                    for (int bb = 0; bb < 2; ++bb) {
+                        uint32_t u[32];
+                        tmem_ld32(lane_base + 32 * (2 * half + bb), r);
+                        tmem_ld32(lane_base + 128 + 32 * (2 * half + bb), u);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const float gv = __uint_as_float(r[i]);
-                                v[32 * c + i] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[i]);
-                            }
-                        } else {
-                            uint32_t r2[32];
-                            tmem_ld32(lane_base + 128 + c0 + 32 * c, r2);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                v[32 * c + i] = __uint_as_float(r[i]);
-                                if (!GU) v2[32 * c + i] = __uint_as_float(r2[i]);
-                            }
+                        for (int i = 0; i < 32; ++i) {
+                            const float gv = __uint_as_float(r[i]);
+                            v[32 * bb + i] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[i]);
                         }
+                    }
+                } else {
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        tmem_ld32(lane_base + 128 * half + 32 * cc, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[32 * cc + i] = __uint_as_float(r[i]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.acc_empty);
+            if (!busy) continue;
             if (GU) {
-                // MXFP8 along F: the block of 32 is this warp's 32 lanes
-                const int fcol = wk.f * kTile + 32 * q + lane;  // this lane's h column
+                // MXFP8 along F: each block of 32 is 32 of this thread's values
                 const int64_t atom = (((int64_t)s.ustart[wk.e] + wk.j) * (a.Nw / kTile) + wk.f) * 512;
-                uint8_t *hrow = a.h8 + (int64_t)(wk.row0 + c0) * a.Nw + fcol;
+                uint8_t *hrow = a.h8 + (int64_t)(wk.row0 + t) * a.Nw + wk.f * kTile + 64 * half;
 #pragma unroll
-                for (int i = 0; i < 64; i += 2) {
-                    if (i >= nc) break;  // warp-uniform
-                    float hv[2];
-                    int se[2];
+                for (int bb = 0; bb < 2; ++bb) {
+                    uint32_t amax = 0;
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        hv[p] = v[i + p];
-                        const uint32_t amax = warp_max_u32(__float_as_uint(hv[p]) & 0x7FFFFFFFu);
-                        if (amax == 0u) {
-                            se[p] = 0;
-                            hv[p] = 0.0f;
-                        } else {
-                            const int e8 = floor_log2_f32(__uint_as_float(amax)) - 8;
-                            se[p] = e8 < -127 ? -127 : (e8 > 127 ? 127 : e8);
-                            hv[p] *= pow2_neg(se[p]);
-                        }
+                    for (int i = 0; i < 32; ++i) amax = max(amax, __float_as_uint(v[32 * bb + i]) & 0x7FFFFFFFu);
+                    int se = 0;
+                    float sc = 0.0f;
+                    if (amax != 0u) {
+                        const int e8 = floor_log2_f32(__uint_as_float(amax)) - 8;
+                        se = e8 < -127 ? -127 : (e8 > 127 ? 127 : e8);
+                        sc = pow2_neg(se);
                     }
-                    const uint32_t codes = f32x2_to_e4m3x2(hv[0], hv[1]);
+                    uint32_t pk[8];
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        if (i + p < nc) {
-                            hrow[(int64_t)(i + p) * a.Nw] = (uint8_t)(codes >> (8 * p));
-                            if (lane == 0) a.hsf[atom + sf_atom_byte(c0 + i + p, q)] = (uint8_t)(se[p] + 127);
-                        }
+                    for (int i = 0; i < 8; ++i)
+                        pk[i] = f32x2_to_e4m3x2(v[32 * bb + 4 * i] * sc, v[32 * bb + 4 * i + 1] * sc) |
+                                f32x2_to_e4m3x2(v[32 * bb + 4 * i + 2] * sc, v[32 * bb + 4 * i + 3] * sc) << 16;
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(hrow + 32 * bb);
+                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        a.hsf[atom + sf_atom_byte(t, 2 * half + bb)] = (uint8_t)(se + 127);
                     }
                 }
-            } else {
-                const int64_t o0 = (int64_t)(wk.row0 + c0) * a.Nw + wk.f * 2 * kTile + 32 * q + lane;
+            } else if (valid) {
+                const int64_t o0 = (int64_t)(wk.row0 + t) * a.Nw + wk.f * 2 * kTile + 128 * half;
                 if (a.out16) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.out16 + o0);
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (i < nc) {
-                            a.out16[o0 + (int64_t)i * a.Nw] = f32_to_bf16_rne(v[i]);
-                            if (!GU) a.out16[o0 + (int64_t)i * a.Nw + kTile] = f32_to_bf16_rne(v2[i]);
-                        }
+                    for (int i = 0; i < 16; ++i)
+                        dst[i] = make_uint4(bf16x2(v[8 * i], v[8 * i + 1]), bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                            bf16x2(v[8 * i + 4], v[8 * i + 5]), bf16x2(v[8 * i + 6], v[8 * i + 7]));
                 } else {
+                    float4 *dst = reinterpret_cast<float4 *>(a.out + o0);
 #pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (i < nc) {
-                            a.out[o0 + (int64_t)i * a.Nw] = v[i];
-                            if (!GU) a.out[o0 + (int64_t)i * a.Nw + kTile] = v2[i];
-                        }
+                    for (int i = 0; i < 32; ++i)
+                        dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                 }
             }
         }
