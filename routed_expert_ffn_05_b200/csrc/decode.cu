@@ -49,22 +49,27 @@ constexpr int kEpilogue = kCW + 1;        // warp index of the epilogue warp
 constexpr int kThreads = (kCW + 2) * 32;
 constexpr int kStageW = 32768;            // weight tile bytes per stage
 // Stages and per-stage scale / metadata bytes by weight format: MXFP4 needs
-// 2 KB of E8M0 per stage, so five stages fit; Q2_K needs 8 KB of sc|m bytes
-// and 2 KB of (d, dmin) and keeps four.
-template <int WF> struct Pipe {
-    static constexpr int stages = WF == MOE_W_Q2K ? 4 : 5;
+// 2 KB of E8M0 per stage, Q2_K 8 KB of sc|m bytes and 2 KB of (d, dmin).
+template <int WF> struct Pipe {  // (five MXFP4 stages were measured: no gain over four)
+    static constexpr int stages = 4;
     static constexpr int meta = WF == MOE_W_Q2K ? 10240 : 2048;
 };
 constexpr int kQDd = 8192;                // Q2_K: offset of the (d, dmin) pairs in a stage's metadata
 constexpr int kMaxE = 1024;
+constexpr int kMaxSeg = 256;              // active experts of a decode batch: min(E, T k) <= 8 x 32
 // Partial tiles: element (matrix m, row r < 16, column c < 8) of a consumer
 // warp's 16x8 tiles at m * 144 + r * 9 + c. One column over all 16 rows and
 // both matrices then falls in 32 different banks (the epilogue reads by
 // column); the consumers' fragment stores conflict at most 2-way.
-constexpr int kRedM = 144, kRedR = 9, kRedW = 2 * kRedM;
+constexpr int kRedM = 144, kRedR = 9;
 constexpr int kD = 4096, kF = 2048;       // the dims this tiling is written for
 constexpr int kGuTiles = kF / 16;         // gate/up tiles per routed expert
-constexpr int kDnTiles = kD / 32;         // down tiles (32 rows) per routed expert
+// A routed down unit: 64 W2 rows over all K (two stages of 32 rows) for
+// MXFP4, 32 rows (one stage) for Q2_K; its partial tiles are 16 rows each.
+template <int WF> constexpr int dn_rows() { return WF == MOE_W_Q2K ? 32 : 64; }
+template <int WF> constexpr int dn_stages() { return dn_rows<WF>() / 32; }
+template <int WF> constexpr int dn_tiles() { return kD / dn_rows<WF>(); }
+template <int WF> constexpr int red_w() { return dn_rows<WF>() / 16 * kRedM; }  // floats per warp
 constexpr int kDshTiles = kD / 16;        // shared-expert down tiles
 
 // Work kinds: shared gate/up (bf16, 8 stages of K 512), routed gate/up (MXFP4,
@@ -95,18 +100,18 @@ struct Smem {
     static constexpr int kStages = Pipe<WF>::stages;
     uint8_t w[kStages][kStageW];
     uint8_t s[kStages][Pipe<WF>::meta];
-    float red[2][kCW][kRedW];    // partial 16x8 tiles per consumer warp (see put_partial)
+    float red[2][kCW][red_w<WF>()];  // partial 16x8 tiles per consumer warp (see put_partial)
     uint64_t full[kStages], empty[kStages], rfull[2], rempty[2];
     int meta_u[kStages], meta_k[kStages];  // unit of the stage, and the unit decoded (pack_unit)
     int rmeta[2];
-    int seg_e[kMaxE];
+    int seg_e[kMaxSeg];
     int n_seg;
     volatile int abort;
     // the epilogue warp's own tables: per active expert its first row, row
     // count and tokens; per token the x prescale
-    int ep_rbase[kMaxE];
-    uint8_t ep_cnt[kMaxE];
-    uint8_t ep_tok[kMaxE][8];
+    int ep_rbase[kMaxSeg];
+    uint8_t ep_cnt[kMaxSeg];
+    uint8_t ep_tok[kMaxSeg][8];
     float ep_xs[8];
 };
 template <int WF> constexpr int smem_bytes() { return (int)sizeof(Smem<WF>) + 1024; }  // + alignment slack
@@ -170,7 +175,7 @@ __device__ __forceinline__ Unit unit_of(int u, int usg, int n_seg, int usd) {
     r -= n_seg * kGuTiles;
     if (r < usd) return Unit{kDsh, -1, r, 2};
     r -= usd;
-    return Unit{kDrt, r / kDnTiles, r % kDnTiles, 1};
+    return Unit{kDrt, r / dn_tiles<WF>(), r % dn_tiles<WF>(), dn_stages<WF>()};
 }
 
 template <class S>
@@ -427,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         auto issue = [&](int u, const Unit &un) {
             int row0 = 0;
             if (un.kind == kGrt) row0 = s.seg_e[un.seg] * kF + 16 * un.tile;
-            if (un.kind == kDrt) row0 = s.seg_e[un.seg] * kD + 32 * un.tile;
+            if (un.kind == kDrt) row0 = s.seg_e[un.seg] * kD + dn_rows<WF>() * un.tile;
             for (int c = 0; c < un.nst && !s.abort; ++c, ++gi) {
                 const int slot = gi % kStages;
                 if (!mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1)) { fail(a, s); return; }
@@ -467,10 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                             tma_load_3d(w, &a.m2c, 0, row0, 0, bar);
                             tma_load_3d(sm, &a.m2s, 0, row0, 0, bar);
                             tma_load_2d(sm + kQDd, &a.m2d, 0, row0, bar);
-                        } else {
+                        } else {  // rows row0 + 32 c .. + 31 of the unit
                             arm(s, slot, u, un, 32768 + 2048);
-                            tma_load_3d(w, &a.m2c, 0, row0, 0, bar);
-                            tma_load_2d(sm, &a.m2s, 0, row0, bar);
+                            tma_load_3d(w, &a.m2c, 0, row0 + 32 * c, 0, bar);
+                            tma_load_2d(sm, &a.m2s, 0, row0 + 32 * c, bar);
                         }
                 }
             }
@@ -482,7 +487,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         }
         __syncwarp();
         grid_dep_wait();  // routing results and zeroed counters from here on
-        const int n = active_experts(a.offsets, a.E, lane, [&](int sg, int e, int, int) { s.seg_e[sg] = e; });
+        const int n = active_experts(a.offsets, a.E, lane, [&](int sg, int e, int, int) {
+            if (sg < kMaxSeg) s.seg_e[sg] = e;
+        });
+        if (n > kMaxSeg) {  // cannot happen for T <= 8, k <= 32; refuse rather than overrun
+            if (lane == 0) fail(a, s);
+            return;
+        }
         if (lane != 0) return;
         s.n_seg = n;
         const int gu_end = usg + n * kGuTiles;
@@ -510,10 +521,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             next = usg + Rs + (int)atomicAdd(a.counters, (uint32_t)kGrab);
             for (int u = u0; u < min(u0 + kGrab, gu_end) && !s.abort; ++u) issue(u, unit_of<WF>(u, usg, n, usd));
         }
-        // this CTA's contiguous share of the down units (shared tiles cost 2 stages)
-        const long long cost = 2ll * usd + (long long)n * kDnTiles;
+        // this CTA's contiguous share of the down units (shared tiles cost 2
+        // stages, routed ones dn_stages)
+        constexpr int kDst = dn_stages<WF>();
+        const long long cost = 2ll * usd + (long long)n * dn_tiles<WF>() * kDst;
         auto first = [&](long long cst) {
-            return gu_end + (cst <= 2ll * usd ? (int)((cst + 1) / 2) : usd + (int)(cst - 2ll * usd));
+            return gu_end + (cst <= 2ll * usd ? (int)((cst + 1) / 2)
+                                              : usd + (int)((cst - 2ll * usd + kDst - 1) / kDst));
         };
         const int d0 = first(cost * blockIdx.x / gridDim.x), d1 = first(cost * (blockIdx.x + 1) / gridDim.x);
         for (int u = d0; u < d1 && !s.abort; ++u) issue(u, unit_of<WF>(u, usg, n, usd));
@@ -537,9 +551,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         grid_dep_wait();
         // per-expert tables, same ascending order as the producer's list
         const int n = active_experts(a.offsets, a.E, lane, [&](int sg, int, int r0, int r1) {
-            s.ep_rbase[sg] = r0;
-            s.ep_cnt[sg] = (uint8_t)(r1 - r0);
+            if (sg < kMaxSeg) {
+                s.ep_rbase[sg] = r0;
+                s.ep_cnt[sg] = (uint8_t)(r1 - r0);
+            }
         });
+        if (n > kMaxSeg) {
+            if (lane == 0) fail(a, s);
+            return;
+        }
         __syncwarp();
         for (int sg = lane; sg < n; sg += 32) {
             const int rb = s.ep_rbase[sg], cnt = s.ep_cnt[sg];
@@ -577,15 +597,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             const Unit un = unit_of<WF>(m >> 3, usg, n, usd);
             // Sum over the consumer warps of one column: lane l takes matrix
             // (or down row half) l / 16, row l % 16 (four chains for latency).
+            constexpr int kRedW = red_w<WF>();
             const float *red = &s.red[rb][0][0] + (lane >> 4) * kRedM + (lane & 15) * kRedR;
-            auto colsum = [&](int c) {
+            auto colsum = [&](int c, int tile_pair = 0) {  // tile pair p: 16-row tiles 2p, 2p + 1
+                const float *rp = red + 2 * kRedM * tile_pair;
                 float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
 #pragma unroll
                 for (int w = 0; w < kCW; w += 4) {
-                    v0 += red[w * kRedW + c];
-                    v1 += red[(w + 1) * kRedW + c];
-                    v2 += red[(w + 2) * kRedW + c];
-                    v3 += red[(w + 3) * kRedW + c];
+                    v0 += rp[w * kRedW + c];
+                    v1 += rp[(w + 1) * kRedW + c];
+                    v2 += rp[(w + 2) * kRedW + c];
+                    v3 += rp[(w + 3) * kRedW + c];
                 }
                 return (v0 + v1) + (v2 + v3);
             };
@@ -628,22 +650,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     float v0 = 0.f, v1 = 0.f;
 #pragma unroll
                     for (int w = 0; w < kCW; w += 2) {
-                        v0 += r0[w * kRedW];
-                        v1 += r0[(w + 1) * kRedW];
+                        v0 += r0[w * red_w<WF>()];
+                        v1 += r0[(w + 1) * red_w<WF>()];
                     }
                     a.shared_out[(int64_t)c * kD + 16 * un.tile + row] = v0 + v1;
                 }
             } else {
-                // lane = row of the 32-row tile; columns = the expert's rows
+                // lane = row of each 32-row part of the unit; columns = the expert's rows
                 const int rbase = s.ep_rbase[un.seg], cnt = s.ep_cnt[un.seg];
                 if (un.seg != dseg) {
                     dseg = un.seg;
                     dsc = lane < cnt ? row_scale(__ldcg(&a.hmax[rbase + lane])) : 1.f;
                 }
-                for (int i = 0; i < cnt; ++i) {
-                    const float sc = __shfl_sync(0xffffffffu, dsc, i);
-                    a.out_rows[(int64_t)(rbase + i) * kD + 32 * un.tile + lane] = colsum(i) * sc;
-                }
+#pragma unroll
+                for (int p = 0; p < dn_stages<WF>(); ++p)
+                    for (int i = 0; i < cnt; ++i) {
+                        const float sc = __shfl_sync(0xffffffffu, dsc, i);
+                        a.out_rows[(int64_t)(rbase + i) * kD + dn_rows<WF>() * un.tile + 32 * p + lane] =
+                            colsum(i, p) * sc;
+                    }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.rempty[rb]);
@@ -833,28 +858,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 release(slot);
             }
         } else {
-            // one stage: 32 W2 rows over all K; rows 16 t + g (+ 8)
-            const uint32_t cw = w_base + (uint32_t)slot * kStageW + 2048u * (uint32_t)(warp >> 1);
-            const uint32_t cs = w_base + kScaleBase + (uint32_t)slot * kStageS + sc_lo;
-            uint32_t sw[2][2];
-            sw[0][0] = lds32_at<0>(cs);
-            sw[0][1] = lds32_at<512>(cs);
-            sw[1][0] = lds32_at<1024>(cs);
-            sw[1][1] = lds32_at<1536>(cs);
+            // dn_stages stages of 32 W2 rows over all K (rows 16 t + g (+ 8) of
+            // each); B (the expert's h rows) is the same for all of them. The
+            // partial tiles go out per stage, so the buffer is claimed first.
+            if (!mbar_wait(&s.rempty[ru & 1], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
+            float *red = s.red[ru & 1][warp];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const uint32_t ad = cw + code_off(code_gu, jj);
-                mxfp4_block<0>(acc[0], ad, sw[0][0], sw[0][1], jj, B[jj]);
-                mxfp4_block<2048>(acc[1], ad, sw[1][0], sw[1][1], jj, B[jj]);
+            for (int c = 0; c < dn_stages<WF>(); ++c) {
+                if (c > 0) {
+                    if (!next_stage()) { fail(a, s); return; }
+#pragma unroll
+                    for (int m = 0; m < 2; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+                }
+                const uint32_t cw = w_base + (uint32_t)slot * kStageW + 2048u * (uint32_t)(warp >> 1);
+                const uint32_t cs = w_base + kScaleBase + (uint32_t)slot * kStageS + sc_lo;
+                uint32_t sw[2][2];
+                sw[0][0] = lds32_at<0>(cs);
+                sw[0][1] = lds32_at<512>(cs);
+                sw[1][0] = lds32_at<1024>(cs);
+                sw[1][1] = lds32_at<1536>(cs);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t ad = cw + code_off(code_gu, jj);
+                    mxfp4_block<0>(acc[0], ad, sw[0][0], sw[0][1], jj, B[jj]);
+                    mxfp4_block<2048>(acc[1], ad, sw[1][0], sw[1][1], jj, B[jj]);
+                }
+                release(slot);
+                put_partial(red + 2 * kRedM * c, g, q, acc[0]);
+                put_partial(red + (2 * c + 1) * kRedM, g, q, acc[1]);
             }
-            release(slot);
         }
-        // hand the unit (or tile) to the epilogue warp
+        // hand the unit (or tile) to the epilogue warp (MXFP4 down units have
+        // put their tiles in place already)
         const int rb = ru & 1;
-        if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
-        const int rg = (un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;  // bf16 tiles read rows sigma(g)
-        put_partial(s.red[rb][warp], rg, q, acc[0]);
-        if (un.kind != kDsh) put_partial(s.red[rb][warp] + kRedM, rg, q, acc[1]);
+        if (Q2 || un.kind != kDrt) {
+            if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
+            const int rg = (un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;  // bf16 tiles read rows sigma(g)
+            put_partial(s.red[rb][warp], rg, q, acc[0]);
+            if (un.kind != kDsh) put_partial(s.red[rb][warp] + kRedM, rg, q, acc[1]);
+        }
         if (threadIdx.x == 0) s.rmeta[rb] = u * 8 + (un.nst - 1);
         __syncwarp();  // the warp's tile stores, then one arrival (release) for the warp
         if (lane == 0) mbar_arrive(&s.rfull[rb]);
