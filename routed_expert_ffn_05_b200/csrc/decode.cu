@@ -1,32 +1,34 @@
 // Decode-sized expert FFN (T <= 8 tokens): one persistent weight-streaming
 // kernel on tensor cores, HBM-bound.
 //
-// Each routed expert is a SwiGLU FFN over MXFP4 weights; the shared expert is
-// bf16 ("DS4", dibi8.com, "Key architectural innovations" item 1; "DwarfStar",
-// hysenlabs.com, "Model support and quantisation"). With at most 8 tokens per
-// expert the layer is a stream over the touched experts' weights, so the
-// kernel is built around keeping HBM busy:
+// Each routed expert is a SwiGLU FFN over MXFP4 (or Q2_K) weights; the shared
+// expert is bf16 ("DS4", dibi8.com, "Key architectural innovations" item 1;
+// "DwarfStar", hysenlabs.com, "Model support and quantisation"). With at most
+// 8 tokens per expert the layer is a stream over the touched experts'
+// weights, so the kernel is built around keeping HBM busy:
 //  - one CTA per SM with three roles: a producer thread moves weight tiles
-//    HBM -> shared memory with TMA (one 16-32 KB tile per instruction,
-//    128-byte swizzled) through four 34 KB mbarrier stages; eight consumer
-//    warps split K and run mma.sync m16n8k16 (16 weight rows x 8 tokens, fp32
-//    accumulate); an epilogue warp reduces the consumers' partial tiles from a
-//    double buffer and writes the outputs, so consumers never wait for one
-//    another;
-//  - gate/up and down run in the same launch: one work queue holds the shared
-//    expert's gate/up tiles, the routed gate/up tiles, then the down tiles,
-//    largest first; a down tile waits (bounded) on a per-expert count of
-//    finished gate/up tiles;
+//    HBM -> shared memory with TMA (16-32 KB boxes, 128-byte swizzled; the
+//    E8M0 scale boxes 64-byte swizzled) through four mbarrier stages; sixteen
+//    consumer warps split K and run mma.sync m16n8k16 (16 weight rows x 8
+//    tokens, fp32 accumulate); an epilogue warp sums the consumers' partial
+//    tiles (double-buffered) and writes the outputs;
+//  - the work is numbered in units (a unit: one or more stages the consumers
+//    run back to back, then one hand-off to the epilogue): shared gate/up
+//    (static per CTA, streamed while routing finishes), routed gate/up (a
+//    cost-balanced static range per CTA plus a dynamic tail from a queue),
+//    then down units as one contiguous static range per CTA; a down unit
+//    waits (bounded) on a per-expert count of finished gate/up tiles;
+//  - the producer stores each stage's decoded unit next to its data, so the
+//    consumers read one word instead of decoding unit numbers;
 //  - MXFP4 codes become f16 with the hardware E2M1 conversion; the E8M0 block
 //    scale is applied per 32-element block in fp32;
 //  - gate/up uses all T tokens as the MMA's N dimension, so its activation
-//    fragments are built once per CTA; outputs for tokens not routed to the
-//    expert are dropped;
+//    fragments are built once per CTA; the epilogue reduces only the columns
+//    of the tokens routed to the expert;
 //  - x enters f16 range through an exact per-token power of two; h, rounded to
 //    bf16 as the layer specifies, gets the same treatment per row from its
 //    maximum, recorded with an order-free atomic max;
-//  - launches are chained with programmatic dependent launch, so the shared
-//    expert's gate/up tiles (which need no routing) stream while routing runs;
+//  - launches are chained with programmatic dependent launch;
 //  - every wait is bounded (MOE_DEVERR_TIMEOUT instead of a hang).
 // K is permuted inside each 32-block identically for weights and activations:
 // lane q of a quad holds elements 8q..8q+7 of a block, which cover its MMA
@@ -74,7 +76,7 @@ constexpr int kDshTiles = kD / 16;        // shared-expert down tiles
 
 // Work kinds: shared gate/up (bf16, 8 stages of K 512), routed gate/up (MXFP4,
 // 2 stages of K 2048), shared down (bf16, 2 stages of K 1024), routed down
-// (MXFP4, one stage: a 32-row tile over all K).
+// (MXFP4: 64 rows over all K in two stages of 32; Q2_K: 32 rows, one stage).
 enum { kGsh = 0, kGrt = 1, kDsh = 2, kDrt = 3 };
 
 struct DecodeArgs {
@@ -679,8 +681,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     // Warp w owns 1/16 of K in every unit: shared gate/up 1 block of 32 per
     // stage (8 stages of K 512), routed MXFP4 gate/up 4 blocks per stage (2 of
     // K 2048), shared down 2 blocks per stage (2 of K 1024), routed MXFP4
-    // down 4 blocks (K 2048), Q2_K gate/up one super-block, Q2_K down half of
-    // one. B holds this warp's activation fragments for the unit's kind.
+    // down 4 blocks of each 32-row stage (K 2048), Q2_K gate/up one
+    // super-block, Q2_K down half of one. B holds this warp's activation
+    // fragments for the unit's kind.
     const int g = lane >> 2, q = lane & 3;
     uint32_t B[8][4];
     uint32_t Bm[4];             // Q2_K: sub-block sums (hi, lo)
