@@ -29,20 +29,25 @@ __global__ void __launch_bounds__(kPermuteBlock) permute_hist_kernel(const int32
     for (int e = threadIdx.x; e < E; e += blockDim.x) blkcnt[(int64_t)blockIdx.x * E + e] = hist[e];
 }
 
-// One block: per-expert running sums over blocks, then the exclusive scan over
-// experts; blkbase[b][e] becomes the first row of block b's slots of expert e.
+// One block: per-expert totals over blocks, the exclusive scan over experts,
+// then blkbase[b][e] = the first row of block b's slots of expert e. Thread e
+// reads its column of block counts 16 at a time (independent loads in flight).
 __global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t *__restrict__ blkcnt,
                                                             int64_t nblk, int E,
                                                             int32_t *__restrict__ blkbase,
                                                             int32_t *__restrict__ counts,
                                                             int32_t *__restrict__ offsets) {
     __shared__ int32_t sc[1024];
+    constexpr int kBatch = 16;
     const int e = threadIdx.x;
     int32_t run = 0;
     if (e < E)
-        for (int64_t b = 0; b < nblk; ++b) {
-            blkbase[b * E + e] = run;
-            run += blkcnt[b * E + e];
+        for (int64_t b0 = 0; b0 < nblk; b0 += kBatch) {
+            int32_t c[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) c[j] = b0 + j < nblk ? blkcnt[(b0 + j) * E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) run += c[j];
         }
     sc[e] = e < E ? run : 0;
     __syncthreads();
@@ -57,7 +62,18 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t *__res
         counts[e] = run;
         offsets[e] = excl;
         if (e == E - 1) offsets[E] = sc[e];
-        for (int64_t b = 0; b < nblk; ++b) blkbase[b * E + e] += excl;
+        int32_t r = excl;
+        for (int64_t b0 = 0; b0 < nblk; b0 += kBatch) {
+            int32_t c[kBatch];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) c[j] = b0 + j < nblk ? blkcnt[(b0 + j) * E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j)
+                if (b0 + j < nblk) {
+                    blkbase[(b0 + j) * E + e] = r;
+                    r += c[j];
+                }
+        }
     }
 }
 
