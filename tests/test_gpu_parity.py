@@ -317,3 +317,21 @@ def test_identical_tokens_identical_outputs():
     M.moe_layer(c.dims, c.weights, dev(x), None, y, c.ws)
     yh = host(y)
     np.testing.assert_array_equal(yh[4], yh[1])
+
+
+@pytest.mark.parametrize("wfmt,T,E", [("mxfp4", 8, 8), ("mxfp4", 3, 16), ("q2k", 8, 8), ("q2k", 5, 16)])
+def test_decode_path_dense_experts(wfmt, T, E):
+    """The fused decode kernel (d 4096, d_ff 2048, shared expert) with few
+    experts: with E = k = 8 every token goes to every expert, so each expert
+    has T rows — the most token columns its gate/up epilogue and its down
+    units handle; E = 16 gives a ragged mix. Every token against the oracle."""
+    from dataclasses import replace
+    cfg = replace(synth.CONFIGS["q2k" if wfmt == "q2k" else "decode"], E=E).with_T(T)
+    c = Case(cfg, experts="all")
+    y = torch.empty((T, cfg.d), dtype=torch.float32, device=DEV)
+    M.moe_layer(c.dims, c.weights, c.x_d, None, y, c.ws)
+    assert M.moe_get_device_error() == 0
+    toks = np.arange(T, dtype=np.int32)
+    idx, _, ref = oracle.layer_tokens(c.ora, c.x, toks)
+    np.testing.assert_array_equal(idx, c.ora_idx)
+    assert_rel(host(y), ref, TOL[cfg.act], f"{wfmt} T={T} E={E}")
