@@ -66,48 +66,61 @@ __device__ __forceinline__ int expert_of_row(const int32_t *offsets, int E, int 
     return lo;
 }
 
-// Ranking key of (logit v, expert e): keys compare as unsigned integers in
-// the routing order -- larger logit first, NaN after every number, ties (and
-// +0 == -0) by the lower expert index. High word: the float made monotone
-// (-0 as +0, NaN as 0); low word: ~e. Key 0 is below every valid key.
-__device__ __forceinline__ uint64_t rank_key(float v, int e) {
+// Routing order of (logit v, expert e): larger logit first, NaN after every
+// number, ties (and +0 == -0) by the lower expert index. rank_word is the
+// float made monotone as an unsigned word (-0 as +0, NaN as 0; every number
+// maps above 0), so the order is: larger word first, then lower index.
+__device__ __forceinline__ uint32_t rank_word(float v) {
     uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
     u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    u = isnan(v) ? 0u : u;
-    return ((uint64_t)u << 32) | (uint32_t)~(uint32_t)e;
+    return isnan(v) ? 0u : u;
 }
-__device__ __forceinline__ int rank_key_expert(uint64_t key) { return (int)~(uint32_t)key; }
 
-// Warp-wide top-k of one row of E <= 1024 logits: lane holds cv[i] = logit of
-// expert lane + 32 i (i < ceil(E / 32)). Round j takes the warp maximum of the
-// unchosen keys; lane j receives pick j in my_e. Callers read the picked
-// logits back by expert index.
-__device__ __forceinline__ int topk_warp(const float (&cv)[32], int E, int k, int lane) {
-    const int nc = (E + 31) >> 5;
-    uint64_t key[32];
+// Warp-wide top-k of one row of E <= 32 NC logits: lane holds cv[i] = logit
+// of expert lane + 32 i. Pick j is the first unchosen expert in routing
+// order, found in two 32-bit warp reductions: the largest rank_word, then the
+// lowest unchosen expert index holding it. Lane j receives pick j. NC is a
+// compile-time bound so the loops stay short (the kernels that use this run
+// once per layer call, from a cold instruction cache).
+template <int NC>
+__device__ __forceinline__ int topk_warp(const float (&cv)[NC], int E, int k, int lane) {
+    uint32_t u[NC], live = 0;  // live: bit i set while expert lane + 32 i is unchosen
 #pragma unroll
-    for (int i = 0; i < 32; ++i) key[i] = (i < nc && lane + 32 * i < E) ? rank_key(cv[i], lane + 32 * i) : 0ull;
+    for (int i = 0; i < NC; ++i) {
+        const bool in = lane + 32 * i < E;
+        u[i] = in ? rank_word(cv[i]) : 0u;
+        live |= in ? 1u << i : 0u;
+    }
     int my_e = -1;
     for (int j = 0; j < k; ++j) {
-        uint64_t best = 0;
+        uint32_t best = 0;  // chosen and absent slots hold 0, at or below every live word
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if (i >= nc) break;  // uniform
-            best = key[i] > best ? key[i] : best;
-        }
+        for (int i = 0; i < NC; ++i) best = max(best, u[i]);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+        uint32_t cand = 0xffffffffu;  // lowest live expert of this lane holding m
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-            best = other > best ? other : best;
-        }
+        for (int i = NC - 1; i >= 0; --i) cand = (u[i] == m && (live >> i & 1u)) ? (uint32_t)(lane + 32 * i) : cand;
+        const int e = (int)__reduce_min_sync(0xffffffffu, cand);
+        if ((e & 31) == lane) live &= ~(1u << (e >> 5));
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if (i >= nc) break;
-            key[i] = key[i] == best ? 0ull : key[i];  // keys are unique: only the pick matches
-        }
-        my_e = lane == j ? rank_key_expert(best) : my_e;
+        for (int i = 0; i < NC; ++i) u[i] = lane + 32 * i == e ? 0u : u[i];
+        my_e = lane == j ? e : my_e;
     }
     return my_e;
+}
+
+// Top-k of the row l[0 .. E) (E <= 1024) by one warp; lane j gets pick j.
+__device__ __forceinline__ int topk_row(const float *l, int E, int k, int lane) {
+    if (E <= 256) {
+        float cv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cv[i] = lane + 32 * i < E ? l[lane + 32 * i] : 0.f;
+        return topk_warp<8>(cv, E, k, lane);
+    }
+    float cv[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) cv[i] = lane + 32 * i < E ? l[lane + 32 * i] : 0.f;
+    return topk_warp<32>(cv, E, k, lane);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -923,6 +923,10 @@ __global__ void __launch_bounds__(256) decode_logits_kernel(const uint16_t *__re
                                                             const float *__restrict__ bias, int T, int E,
                                                             float *__restrict__ logits, float2 *__restrict__ xscale) {
     __shared__ uint4 ws4[16 * 32];
+    // the finalize kernel (and through it the FFN kernel, whose shared-expert
+    // tiles need no routing) may launch at once: they wait for this grid
+    // before reading anything it writes
+    grid_dep_launch();
     const int t = threadIdx.x >> 5, lane = threadIdx.x & 31, e = blockIdx.x;
     constexpr int chunk = kD / 32;  // 128 elements = 16 uint4 per lane
     for (int i = threadIdx.x; i < 16 * 32; i += blockDim.x)
@@ -932,7 +936,6 @@ __global__ void __launch_bounds__(256) decode_logits_kernel(const uint16_t *__re
     for (int v = 0; v < 16; ++v) xv[v] = ldg128(x + (int64_t)t * kD + lane * chunk + 8 * v);
     cp_async_wait_all();
     __syncthreads();
-    grid_dep_launch();
     if (e == 0) {  // 2^p with max|x_t| 2^-p in [2^14, 2^15)
         float mx = 0.f;
 #pragma unroll
@@ -1002,10 +1005,7 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
     __syncthreads();
     if (warp < T) {  // top-k + gates of token `warp`: lane holds experts lane + 32 i
         const float *l = lg + warp * E;
-        float cv[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) cv[i] = lane + 32 * i < E ? l[lane + 32 * i] : 0.f;
-        const int my_e = topk_warp(cv, E, k, lane);
+        const int my_e = topk_row(l, E, k, lane);
         const float my_l = lane < k ? l[my_e] : 0.f;
         const float l0v = __shfl_sync(0xffffffffu, my_l, 0);
         const float ex = lane < k ? expf(my_l - l0v) : 0.f;

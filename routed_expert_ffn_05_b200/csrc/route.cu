@@ -163,10 +163,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float *__restri
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (t >= T) return;
     const float *l = logits + (int64_t)t * E;
-    float cv[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) cv[i] = lane + 32 * i < E ? l[lane + 32 * i] : 0.f;
-    const int my_e = topk_warp(cv, E, k, lane);
+    const int my_e = topk_row(l, E, k, lane);
     const float my_l = lane < k ? l[my_e] : 0.f;
     const float l0 = __shfl_sync(0xffffffffu, my_l, 0);
     const float ex = lane < k ? expf(my_l - l0) : 0.0f;

@@ -67,13 +67,15 @@ def host_weights(cfg, seed=0) -> HostWeights:
 class Case:
     """A layer config with its seeded inputs on host and device."""
 
-    def __init__(self, cfg, seed=0, batch=0, experts="routed"):
+    def __init__(self, cfg, seed=0, batch=0, experts="routed", router_fn=None):
         import torch
         import routed_expert_ffn_05_b200 as M
         self.M, self.cfg, self.seed = M, cfg, seed
         self.x = synth.make_x(cfg, seed, batch)
         self.token_ids = synth.make_token_ids(cfg, seed, batch) if cfg.route == "hash" else None
         self.wr = synth.make_router(cfg, seed) if cfg.has_router else None
+        if router_fn is not None:  # a test's edit of the router rows (ties and the like)
+            router_fn(self.wr)
         self.bias = synth.make_bias(cfg, seed)
         self.shared = synth.shared_weights_bf16(cfg, seed)
         self.hw = host_weights(cfg, seed)

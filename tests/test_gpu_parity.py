@@ -319,6 +319,35 @@ def test_identical_tokens_identical_outputs():
     np.testing.assert_array_equal(yh[4], yh[1])
 
 
+def test_decode_route_ties_to_lower_index():
+    """The decode layer's own routing kernels break ties by the lower expert
+    index. Token 0's last pick a shares its router row with the two lowest
+    experts token 0 leaves out, so the three tie bit for bit at token 0's
+    k-th place and only the lowest of them may be taken. Each expert has its
+    own weights, so another pick shows in y."""
+    from dataclasses import replace
+    cfg = replace(synth.CONFIGS["decode"], E=16).with_T(8)
+    assert synth.make_bias(cfg, 0) is None
+    idx0, _ = oracle.topk_softmax(oracle.router_logits(synth.make_x(cfg, 0, 0), synth.make_router(cfg, 0)), cfg.k)
+    a = int(idx0[0, -1])
+    b, c = [e for e in range(cfg.E) if e not in idx0[0]][:2]
+
+    def tie(wr):
+        wr[b] = wr[a]
+        wr[c] = wr[a]
+
+    case = Case(cfg, experts="all", router_fn=tie)
+    assert len({a, b, c} & set(case.ora_idx[0].tolist())) == 1
+    assert min(a, b, c) in case.ora_idx[0]
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device=DEV)
+    M.moe_layer(case.dims, case.weights, case.x_d, None, y, case.ws)
+    assert M.moe_get_device_error() == 0
+    toks = np.arange(cfg.T, dtype=np.int32)
+    idx, _, ref = oracle.layer_tokens(case.ora, case.x, toks)
+    np.testing.assert_array_equal(idx, case.ora_idx)
+    assert_rel(host(y), ref, TOL[cfg.act], "decode ties")
+
+
 @pytest.mark.parametrize("wfmt,T,E", [("mxfp4", 8, 8), ("mxfp4", 3, 16), ("q2k", 8, 8), ("q2k", 5, 16)])
 def test_decode_path_dense_experts(wfmt, T, E):
     """The fused decode kernel (d 4096, d_ff 2048, shared expert) with few
