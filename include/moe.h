@@ -29,7 +29,8 @@
  *    MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED and launches nothing.
  *  - Errors found by a kernel (an expert index outside [0, E), hash routing
  *    that needs more than 1024 draws for one token, a bounded wait that gave
- *    up) set a per-device error word; the outputs of that call are then
+ *    up, a perm that is not a permutation of the T*k slots) set a per-device
+ *    error word; the outputs of that call are then
  *    undefined. Read and clear it with moe_get_device_error.
  *  - bf16 values travel as uint16_t bit patterns. Row-major everywhere.
  *  - Calls on distinct workspaces may run concurrently; weights are read-only.
@@ -69,7 +70,7 @@ typedef enum { MOE_ROUTE_SOFTMAX_TOPK = 0, MOE_ROUTE_HASH = 1 } moe_rmode;
 
 /* Device error codes (moe_get_device_error). */
 enum { MOE_DEVERR_NONE = 0, MOE_DEVERR_EXPERT_RANGE = 1, MOE_DEVERR_HASH_CAP = 2,
-       MOE_DEVERR_TIMEOUT = 3 };
+       MOE_DEVERR_TIMEOUT = 3, MOE_DEVERR_PERM = 4 };
 
 /* Layer shape. Limits: d_model and d_ff multiples of 256 (of 32 for MXFP4),
  * 1 <= k <= min(E, 32), E <= 1024, T*k < 2^31. */
@@ -156,7 +157,9 @@ MOE_API moe_status moe_permute(const moe_dims *dims, const int32_t *topk_idx, in
 
 /* Routed expert FFNs for every permuted row: out_rows fp32 [T*k][d_model],
  * row r = o_{e}(x[perm[r] / k]) for the expert e whose segment holds r.
- * x bf16 [T][d_model]. In MXFP8 mode x and h are quantised on the fly. */
+ * x bf16 [T][d_model]. perm is a permutation of 0 .. T*k-1, as moe_permute
+ * writes it (the MXFP8 path checks this: MOE_DEVERR_PERM otherwise). In MXFP8
+ * mode x and h are quantised on the fly. */
 MOE_API moe_status moe_expert_ffn(const moe_dims *dims, const moe_weights *weights, const uint16_t *x,
                           const int32_t *offsets, const int32_t *perm, float *out_rows, void *ws,
                           void *stream);

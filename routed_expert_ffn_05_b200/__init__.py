@@ -22,7 +22,7 @@ MOE_W_MXFP4, MOE_W_Q2K = 1, 2
 MOE_A_BF16, MOE_A_MXFP8 = 0, 1
 MOE_ROUTE_SOFTMAX_TOPK, MOE_ROUTE_HASH = 0, 1
 MOE_MAT_W1, MOE_MAT_W2, MOE_MAT_W3 = 1, 2, 3
-MOE_DEVERR_NONE, MOE_DEVERR_EXPERT_RANGE, MOE_DEVERR_HASH_CAP, MOE_DEVERR_TIMEOUT = range(4)
+MOE_DEVERR_NONE, MOE_DEVERR_EXPERT_RANGE, MOE_DEVERR_HASH_CAP, MOE_DEVERR_TIMEOUT, MOE_DEVERR_PERM = range(5)
 
 
 class MoeError(RuntimeError):

@@ -76,7 +76,7 @@ static inline Q2kLayout q2k_layout(const moe_dims &d, int which) {
 struct WsLayout {
     int64_t logits, topk_idx, topk_w, counts, offsets, perm, inv_perm, blkcnt, blkbase;
     int64_t x8, xs, xscale, counters, h, hmax, h8, hs, out_rows, sh_h, sh_out;
-    int64_t ustart, gx8, gxsf, ghsf, total;
+    int64_t ustart, row_of, gx8, gxsf, ghsf, total;
     int64_t nblk, max_tiles;
 };
 static const int kPermuteBlock = 256;  // slots per permute block
@@ -109,10 +109,11 @@ static inline WsLayout ws_layout(const moe_dims &d) {
     w.sh_h = take(T * Fs * 4);
     w.sh_out = take(T * dm * 4);
     // tensor-core path: token tiles of 128 rows per expert (at most
-    // ceil(S / 128) + E of them), gathered MXFP8 rows, and scale atoms of
-    // 512 bytes per (token tile, 128-wide K block)
+    // ceil(S / 128) + E of them), the slot -> row inverse of perm, gathered
+    // MXFP8 rows, and scale atoms of 512 bytes per (token tile, 128-wide K block)
     w.max_tiles = (S + 127) / 128 + E;
     w.ustart = take((E + 1) * 4);
+    w.row_of = take(S * 4);  // slot -> permuted row
     w.gx8 = take(S * dm);
     w.gxsf = take(w.max_tiles * (dm / 128) * 512);
     w.ghsf = take(w.max_tiles * (F / 128) * 512);

@@ -30,51 +30,68 @@ __global__ void __launch_bounds__(kPermuteBlock) permute_hist_kernel(const int32
 }
 
 // One block: per-expert totals over blocks, the exclusive scan over experts,
-// then blkbase[b][e] = the first row of block b's slots of expert e. Thread e
-// reads its column of block counts 16 at a time (independent loads in flight).
+// then blkbase[b][e] = the first row of block b's slots of expert e. The
+// 1024 threads are G = 1024 / ep groups of ep (E rounded up to a power of
+// two): thread (g, e) owns expert e's counts in the g-th contiguous range of
+// blocks and reads them 16 at a time, once for its partial sum and once to
+// write the bases (consecutive threads read consecutive experts of a block).
 __global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t *__restrict__ blkcnt,
                                                             int64_t nblk, int E,
                                                             int32_t *__restrict__ blkbase,
                                                             int32_t *__restrict__ counts,
                                                             int32_t *__restrict__ offsets) {
+    __shared__ int32_t part[1024];  // [g][e]: partial sums, then the group's first row
     __shared__ int32_t sc[1024];
     constexpr int kBatch = 16;
-    const int e = threadIdx.x;
+    int ep = 1;
+    while (ep < E) ep <<= 1;
+    const int G = 1024 / ep, e = threadIdx.x % ep, g = threadIdx.x / ep;
+    const int64_t b_lo = nblk * g / G, b_hi = nblk * (g + 1) / G;
+    const bool own = e < E;
     int32_t run = 0;
-    if (e < E)
-        for (int64_t b0 = 0; b0 < nblk; b0 += kBatch) {
+    if (own)
+        for (int64_t b0 = b_lo; b0 < b_hi; b0 += kBatch) {
             int32_t c[kBatch];
 #pragma unroll
-            for (int j = 0; j < kBatch; ++j) c[j] = b0 + j < nblk ? blkcnt[(b0 + j) * E + e] : 0;
+            for (int j = 0; j < kBatch; ++j) c[j] = b0 + j < b_hi ? blkcnt[(b0 + j) * E + e] : 0;
 #pragma unroll
             for (int j = 0; j < kBatch; ++j) run += c[j];
         }
-    sc[e] = e < E ? run : 0;
+    part[threadIdx.x] = run;
     __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {  // inclusive Hillis-Steele scan
-        const int32_t v = e >= o ? sc[e - o] : 0;
+    int32_t tot = 0;  // thread i < ep: expert i's total
+    if (threadIdx.x < ep)
+        for (int gg = 0; gg < G; ++gg) tot += part[gg * ep + threadIdx.x];
+    sc[threadIdx.x] = tot;
+    __syncthreads();
+    for (int o = 1; o < ep; o <<= 1) {  // inclusive Hillis-Steele scan over the experts
+        const int32_t v = threadIdx.x < ep && threadIdx.x >= o ? sc[threadIdx.x - o] : 0;
         __syncthreads();
-        sc[e] += v;
+        sc[threadIdx.x] += v;
         __syncthreads();
     }
-    if (e < E) {
-        const int32_t excl = sc[e] - run;
-        counts[e] = run;
-        offsets[e] = excl;
-        if (e == E - 1) offsets[E] = sc[e];
-        int32_t r = excl;
-        for (int64_t b0 = 0; b0 < nblk; b0 += kBatch) {
+    if (threadIdx.x < E) {
+        counts[threadIdx.x] = tot;
+        offsets[threadIdx.x] = sc[threadIdx.x] - tot;
+        if (threadIdx.x == E - 1) offsets[E] = sc[threadIdx.x];
+    }
+    int32_t r = 0;  // first row of this group's slots of expert e
+    if (own) {
+        r = e > 0 ? sc[e - 1] : 0;
+        for (int gg = 0; gg < g; ++gg) r += part[gg * ep + e];
+    }
+    if (own)
+        for (int64_t b0 = b_lo; b0 < b_hi; b0 += kBatch) {
             int32_t c[kBatch];
 #pragma unroll
-            for (int j = 0; j < kBatch; ++j) c[j] = b0 + j < nblk ? blkcnt[(b0 + j) * E + e] : 0;
+            for (int j = 0; j < kBatch; ++j) c[j] = b0 + j < b_hi ? blkcnt[(b0 + j) * E + e] : 0;
 #pragma unroll
             for (int j = 0; j < kBatch; ++j)
-                if (b0 + j < nblk) {
+                if (b0 + j < b_hi) {
                     blkbase[(b0 + j) * E + e] = r;
                     r += c[j];
                 }
         }
-    }
 }
 
 __global__ void __launch_bounds__(kPermuteBlock) permute_scatter_kernel(

@@ -337,9 +337,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     }
 }
 
-// Token tiles per expert (ceil(count / 128)) and their exclusive prefix.
+// CTA 0: token tiles per expert (ceil(count / 128)) and their exclusive
+// prefix. The other CTAs invert perm: row_of[slot] = the row holding the slot
+// (row_of enters filled with -1, so a slot no row names stays -1).
 __global__ void __launch_bounds__(1024) tc_plan_kernel(const int32_t *__restrict__ offsets, int E,
-                                                       int32_t *__restrict__ ustart) {
+                                                       int32_t *__restrict__ ustart,
+                                                       const int32_t *__restrict__ perm, int S,
+                                                       int32_t *__restrict__ row_of, int *err) {
+    if (blockIdx.x > 0) {
+        const int i = (blockIdx.x - 1) * blockDim.x + threadIdx.x;
+        if (i < S) {
+            const int slot = perm[i];
+            if ((unsigned)slot < (unsigned)S) row_of[slot] = i;
+            else set_device_error(err, MOE_DEVERR_PERM);
+        }
+        return;
+    }
     __shared__ int wsum[32];
     const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
     const int nt = e < E ? (offsets[e + 1] - offsets[e] + kTile - 1) / kTile : 0;
@@ -366,52 +379,73 @@ __global__ void __launch_bounds__(1024) tc_plan_kernel(const int32_t *__restrict
     if (e == E - 1) ustart[E] = excl + nt;
 }
 
-// One warp per permuted row: x of the row's token -> MXFP8 (E4M3 codes and
-// E8M0 scales per 32 along d, the OCP rule: scale exponent floor(log2 amax) - 8,
-// RNE, saturating; an all-zero block gets scale 127 and zero codes). Codes go
-// to the row in expert order, scales to the row's token-tile atom.
+// One warp per token: its x row becomes MXFP8 once (E4M3 codes and E8M0
+// scales per 32 along d, the OCP rule: scale exponent floor(log2 amax) - 8,
+// RNE, saturating; an all-zero block gets scale 127 and zero codes), and the
+// codes go to each of the token's k rows in expert order, the scales to those
+// rows' token-tile atoms. x is read once per token instead of once per row.
 __global__ void __launch_bounds__(256) tc_gather_quant_kernel(const uint16_t *__restrict__ x,
                                                               const int32_t *__restrict__ offsets,
-                                                              const int32_t *__restrict__ perm,
-                                                              const int32_t *__restrict__ ustart, int S, int E,
+                                                              const int32_t *__restrict__ row_of,
+                                                              const int32_t *__restrict__ ustart, int T, int E,
                                                               int k, int d, uint8_t *__restrict__ x8,
-                                                              uint8_t *__restrict__ xsf) {
-    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (row >= S) return;
-    const int e = expert_of_row(offsets, E, row);
-    const int r = row - offsets[e];
-    const int tok = perm[row] / k;
-    const int64_t atom0 = ((int64_t)ustart[e] + r / kTile) * (d / kTile);
-    const uint16_t *xr = x + (int64_t)tok * d;
-    for (int c = 0; c < d; c += 256) {
-        const int i0 = c + 8 * lane;
-        const bool in = i0 < d;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (in) v = __ldg(reinterpret_cast<const uint4 *>(xr + i0));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float f[8], amax = 0.0f;
+                                                              uint8_t *__restrict__ xsf, int *err) {
+    __shared__ int s_row[8][32], s_rt[8][32];
+    __shared__ int64_t s_atom[8][32];
+    const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + wl;
+    if (t >= T) return;
+    const int S = T * k;
+    if (lane < k) {  // slot (t, lane): its row, the row's token-tile atom base and place in the tile
+        int row = row_of[(int64_t)t * k + lane];
+        if ((unsigned)row >= (unsigned)S) {
+            set_device_error(err, MOE_DEVERR_PERM);
+            row = -1;
+        } else {
+            const int e = expert_of_row(offsets, E, row), r = row - offsets[e];
+            s_atom[wl][lane] = ((int64_t)ustart[e] + r / kTile) * (d / kTile);
+            s_rt[wl][lane] = r % kTile;
+        }
+        s_row[wl][lane] = row;
+    }
+    __syncwarp();
+    const uint16_t *xr = x + (int64_t)t * d;
+    for (int c0 = 0; c0 < d; c0 += 4 * 256) {
+        uint4 v[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            f[2 * i] = __uint_as_float(w[i] << 16);
-            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-            amax = fmaxf(amax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
+        for (int u = 0; u < 4; ++u) {  // four loads in flight
+            const int i0 = c0 + 256 * u + 8 * lane;
+            v[u] = i0 < d ? __ldg(reinterpret_cast<const uint4 *>(xr + i0)) : make_uint4(0, 0, 0, 0);
         }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        uint32_t lo = 0, hi = 0, sb = 127;
-        if (amax > 0.0f) {
-            int se = floor_log2_f32(amax) - 8;
-            se = se < -127 ? -127 : (se > 127 ? 127 : se);
-            sb = (uint32_t)(se + 127);
-            const float sc = pow2_neg(se);
-            lo = f32x2_to_e4m3x2(f[0] * sc, f[1] * sc) | f32x2_to_e4m3x2(f[2] * sc, f[3] * sc) << 16;
-            hi = f32x2_to_e4m3x2(f[4] * sc, f[5] * sc) | f32x2_to_e4m3x2(f[6] * sc, f[7] * sc) << 16;
-        }
-        if (in) {
-            *reinterpret_cast<uint2 *>(x8 + (int64_t)row * d + i0) = make_uint2(lo, hi);
-            if ((lane & 3) == 0) {
-                const int b = i0 / 32;
-                xsf[(atom0 + b / 4) * 512 + sf_atom_byte(r % kTile, b % 4)] = (uint8_t)sb;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i0 = c0 + 256 * u + 8 * lane;
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            float f[8], amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                f[2 * i] = __uint_as_float(w[i] << 16);
+                f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+                amax = fmaxf(amax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
+            }
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            uint32_t lo = 0, hi = 0, sb = 127;
+            if (amax > 0.0f) {
+                int se = floor_log2_f32(amax) - 8;
+                se = se < -127 ? -127 : (se > 127 ? 127 : se);
+                sb = (uint32_t)(se + 127);
+                const float sc = pow2_neg(se);
+                lo = f32x2_to_e4m3x2(f[0] * sc, f[1] * sc) | f32x2_to_e4m3x2(f[2] * sc, f[3] * sc) << 16;
+                hi = f32x2_to_e4m3x2(f[4] * sc, f[5] * sc) | f32x2_to_e4m3x2(f[6] * sc, f[7] * sc) << 16;
+            }
+            if (i0 >= d) continue;
+            const int b = i0 / 32;
+            for (int j = 0; j < k; ++j) {
+                const int row = s_row[wl][j];
+                if (row < 0) continue;
+                *reinterpret_cast<uint2 *>(x8 + (int64_t)row * d + i0) = make_uint2(lo, hi);
+                if ((lane & 3) == 0) xsf[(s_atom[wl][j] + b / 4) * 512 + sf_atom_byte(s_rt[wl][j], b % 4)] = (uint8_t)sb;
             }
         }
     }
@@ -480,8 +514,11 @@ cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_
     else dn.out = out_rows;
     dn.err = g.err;
 
-    tc_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.E, ustart);
-    tc_gather_quant_kernel<<<(S + 7) / 8, 256, 0, s>>>(x, offsets, perm, ustart, S, d.E, d.k, d.d_model, gx8, gxsf);
+    int32_t *row_of = reinterpret_cast<int32_t *>(ws + L.row_of);
+    if ((e = cudaMemsetAsync(row_of, 0xFF, (size_t)S * 4, s)) != cudaSuccess) return e;
+    tc_plan_kernel<<<1 + (S + 1023) / 1024, 1024, 0, s>>>(offsets, d.E, ustart, perm, S, row_of, g.err);
+    tc_gather_quant_kernel<<<(d.T + 7) / 8, 256, 0, s>>>(x, offsets, row_of, ustart, d.T, d.E, d.k, d.d_model, gx8,
+                                                         gxsf, g.err);
     const int grid = tc_num_sms();
     tc_ffn_kernel<kModeGU><<<grid, kTcThreads, kTcSmemBytes, s>>>(g);
     tc_ffn_kernel<kModeDN><<<grid, kTcThreads, kTcSmemBytes, s>>>(dn);

@@ -308,6 +308,27 @@ def test_expert_ffn_w4a8_every_row(T, k, E):
     assert_rel(host(out), ref, TOL["mxfp8"], f"w4a8 T={T} k={k} E={E}")
 
 
+@pytest.mark.parametrize("bad", ["duplicate", "out_of_range"])
+def test_expert_ffn_w4a8_bad_perm_sets_device_error(bad):
+    """The w4a8 path inverts perm to quantise each token once; a perm that is
+    not a permutation of the T*k slots is reported, not followed."""
+    cfg = synth.LayerConfig("w4a8", T=37, d=256, F=512, E=8, k=2, act="mxfp8")
+    c = Case(cfg, experts="all")
+    _, offsets_r, perm_r, _ = oracle.permute(c.ora_idx, cfg.E)
+    perm_bad = perm_r.copy()
+    if bad == "duplicate":
+        perm_bad[5] = perm_bad[4]
+    else:
+        perm_bad[3] = cfg.T * cfg.k + 5
+    out = torch.empty((cfg.T * cfg.k, cfg.d), dtype=torch.float32, device=DEV)
+    M.moe_expert_ffn(c.dims, c.weights, c.x_d, dev(offsets_r), dev(perm_bad), out, c.ws)
+    assert M.moe_get_device_error() == M.MOE_DEVERR_PERM
+    M.moe_expert_ffn(c.dims, c.weights, c.x_d, dev(offsets_r), dev(perm_r), out, c.ws)
+    assert M.moe_get_device_error() == 0   # the next good call is clean
+    ref = oracle.expert_ffn_rows(c.ora, c.x, offsets_r, perm_r, 0, cfg.T * cfg.k)
+    assert_rel(host(out), ref, TOL["mxfp8"], f"w4a8 after bad perm ({bad})")
+
+
 def test_identical_tokens_identical_outputs():
     cfg = synth.LayerConfig("dup", T=6, d=256, F=512, E=8, k=2)
     c = Case(cfg, experts="all")
