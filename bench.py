@@ -145,6 +145,37 @@ def algorithmic_ffn_bytes(cfg, n_experts_touched):
     return per * n_experts_touched + 3 * cfg.Fs * cfg.d * 2
 
 
+# DRAM traffic of one decode_ffn_kernel launch on batch 0 of the default
+# workload (decode T=8, 256 experts, 58 of them touched): dram__bytes_read.sum +
+# dram__bytes_write.sum from a one-pass ncu capture of that launch (826.33 +
+# 4.47 MB as ncu printed them; command and figures in
+# profiles/decode_ffn_kernel_traffic_decode_T8.md). The figure belongs to the
+# sources it was taken on: their SHA-256 is checked before it is reported.
+DECODE_TRAFFIC = {
+    "T": 8, "E": 256, "dram_bytes": 830_800_000,
+    "sources": ["routed_expert_ffn_05_b200/csrc/decode.cu", "routed_expert_ffn_05_b200/csrc/common.cuh",
+                "routed_expert_ffn_05_b200/csrc/kernels.h", "routed_expert_ffn_05_b200/csrc/ptx.cuh",
+                "routed_expert_ffn_05_b200/csrc/tma.h", "routed_expert_ffn_05_b200/csrc/tma.cu",
+                "routed_expert_ffn_05_b200/csrc/layout.h", "include/moe.h"],
+    "sources_sha256": "d8dad1616d9e0f2d1e26667a34b0d83a67afe39cecd892a08e98ddf7852e90d4",
+}
+
+
+def decode_traffic(cfg, T):
+    """The captured per-launch DRAM bytes when this run is that workload on the
+    captured sources, else None."""
+    rec = DECODE_TRAFFIC
+    if not (cfg.wfmt == "mxfp4" and cfg.act == "bf16" and cfg.route == "softmax" and T == rec["T"]
+            and cfg.E == rec["E"] and cfg.d == 4096 and cfg.F == 2048 and cfg.Fs == 2048):
+        return None
+    import hashlib
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return rec["dram_bytes"] if h.hexdigest() == rec["sources_sha256"] else None
+
+
 def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=False):
     """Times `steps` moe_layer calls; returns a dict of per-step times (ms)."""
     cfg = layer.cfg
@@ -442,7 +473,7 @@ def main():
         achieved = alg / (ffn_ms / 1000.0) / 1e9
         roof = {"kernel": "expert FFN: routed + shared", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_source": src, "traffic": None,
+                "peak_source": src, "traffic": decode_traffic(cfg, T),
                 "algorithmic_bytes": alg, "experts_touched": U, "ffn_ms": ffn_ms}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
