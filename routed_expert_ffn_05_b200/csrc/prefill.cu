@@ -250,25 +250,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             tc_fence_after();
             const bool busy = 32 * q < wk.nvalid;  // warp-uniform: any valid token in this quarter
             const bool valid = t < wk.nvalid;
-            // Pull this warp's columns out of TMEM (gate/up: h = silu(g) u right
-            // away), then hand the accumulator back before the slow part, so the
-            // next tile's MMAs overlap the requantisation and the stores.
+            // Pull this warp's columns out of TMEM (gate/up: its g and u columns,
+            // four loads and one wait), then hand the accumulator back before the
+            // slow part, so the next tile's MMAs overlap the SwiGLU, the
+            // requantisation and the stores.
             float v[GU ? 64 : 128];
+            uint32_t g0[32], g1[32], u0[32], u1[32];  // gate/up: raw g, u; then h in g0, g1
             if (busy) {
                 uint32_t r[32];
                 if (GU) {
-#pragma unroll
-                    for (int bb = 0; bb < 2; ++bb) {
-                        uint32_t u[32];
-                        tmem_ld32(lane_base + 32 * (2 * half + bb), r);
-                        tmem_ld32(lane_base + 128 + 32 * (2 * half + bb), u);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float gv = __uint_as_float(r[i]);
-                            v[32 * bb + i] = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[i]);
-                        }
-                    }
+                    tmem_ld32(lane_base + 32 * (2 * half), g0);
+                    tmem_ld32(lane_base + 32 * (2 * half + 1), g1);
+                    tmem_ld32(lane_base + 128 + 32 * (2 * half), u0);
+                    tmem_ld32(lane_base + 128 + 32 * (2 * half + 1), u1);
+                    tmem_wait_ld();
                 } else {
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc) {
@@ -284,6 +279,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             if (lane == 0) mbar_arrive(&s.acc_empty);
             if (!busy) continue;
             if (GU) {
+                // h = silu(g) u, in place (fewer live registers than a separate array)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float ga = __uint_as_float(g0[i]), gb = __uint_as_float(g1[i]);
+                    g0[i] = __float_as_uint(__fdividef(ga, 1.0f + __expf(-ga)) * __uint_as_float(u0[i]));
+                    g1[i] = __float_as_uint(__fdividef(gb, 1.0f + __expf(-gb)) * __uint_as_float(u1[i]));
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    v[i] = __uint_as_float(g0[i]);
+                    v[32 + i] = __uint_as_float(g1[i]);
+                }
                 // MXFP8 along F: each block of 32 is 32 of this thread's values
                 const int64_t atom = (((int64_t)s.ustart[wk.e] + wk.j) * (a.Nw / kTile) + wk.f) * 512;
                 uint8_t *hrow = a.h8 + (int64_t)(wk.row0 + t) * a.Nw + wk.f * kTile + 64 * half;
