@@ -250,27 +250,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             tc_fence_after();
             const bool busy = 32 * q < wk.nvalid;  // warp-uniform: any valid token in this quarter
             const bool valid = t < wk.nvalid;
-            // Pull this warp's columns out of TMEM (gate/up: its g and u columns,
-            // four loads and one wait), then hand the accumulator back before the
-            // slow part, so the next tile's MMAs overlap the SwiGLU, the
-            // requantisation and the stores.
+            // Pull this warp's columns out of TMEM (four loads and one wait; gate/up:
+            // its g and u columns), then hand the accumulator back before the slow
+            // part, so the next tile's MMAs overlap the SwiGLU, the requantisation
+            // and the stores.
             float v[GU ? 64 : 128];
-            uint32_t g0[32], g1[32], u0[32], u1[32];  // gate/up: raw g, u; then h in g0, g1
+            uint32_t g0[32], g1[32], u0[32], u1[32];  // gate/up: raw g, u, then h in g0, g1
             if (busy) {
-                uint32_t r[32];
                 if (GU) {
                     tmem_ld32(lane_base + 32 * (2 * half), g0);
                     tmem_ld32(lane_base + 32 * (2 * half + 1), g1);
                     tmem_ld32(lane_base + 128 + 32 * (2 * half), u0);
                     tmem_ld32(lane_base + 128 + 32 * (2 * half + 1), u1);
                     tmem_wait_ld();
-                } else {
+                } else {  // the tile's four 32-column chunks of this warp's 128 features
+                    tmem_ld32(lane_base + 128 * half, g0);
+                    tmem_ld32(lane_base + 128 * half + 32, g1);
+                    tmem_ld32(lane_base + 128 * half + 64, u0);
+                    tmem_ld32(lane_base + 128 * half + 96, u1);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        tmem_ld32(lane_base + 128 * half + 32 * cc, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[32 * cc + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 32; ++i) {
+                        v[i] = __uint_as_float(g0[i]);
+                        v[32 + i] = __uint_as_float(g1[i]);
+                        v[64 + i] = __uint_as_float(u0[i]);
+                        v[96 + i] = __uint_as_float(u1[i]);
                     }
                 }
             }
