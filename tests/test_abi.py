@@ -61,3 +61,42 @@ def test_host_side_argument_checks():
         M.moe_route(M.make_dims(4, 4096, 2048, 256, 8, route=M.MOE_ROUTE_HASH), 0x1000, w, None,
                     0x1000, 0x1000, 0x1000, stream=0)
     assert M.status_string(M.MOE_ERR_DEVICE) == "device error word set"
+
+
+def header_constants():
+    """Every `MOE_NAME = value` an enum of the header defines."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for body in re.findall(r"enum\s*\{(.*?)\}", src, flags=re.S):
+        for name, val in re.findall(r"(MOE_\w+)\s*=\s*(\d+)", body):
+            out[name] = int(val)
+    return out
+
+
+def header_struct_fields(name):
+    """Field names of `typedef struct { ... } name;` in declaration order."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    body = re.search(r"typedef struct\s*\{([^}]*)\}\s*" + name + r"\s*;", src).group(1)
+    fields = []
+    for decl in body.split(";"):
+        for part in decl.split(","):
+            words = re.findall(r"\w+", part)
+            if words:
+                fields.append(words[-1])
+    return fields
+
+
+def test_binding_constants_match_the_header():
+    import routed_expert_ffn_05_b200 as M
+    consts = header_constants()
+    assert len(consts) >= 20
+    for name, val in consts.items():
+        assert getattr(M, name) == val, name
+
+
+def test_binding_structs_match_the_header():
+    import routed_expert_ffn_05_b200 as M
+    assert [f for f, _ in M.moe_dims._fields_] == header_struct_fields("moe_dims")
+    assert [f for f, _ in M.moe_weights._fields_] == header_struct_fields("moe_weights")
