@@ -132,6 +132,21 @@ def test_splitmix_increment_is_golden_ratio_constant(ora):
     assert a[1:] == b
 
 
+def test_splitmix_outputs_match_a_library_splitmix64(ora):
+    """numba's xoroshiro128+ seeding is a library implementation of the
+    SplitMix64 generator's first output (state + golden-ratio increment, then
+    the finaliser). Output j for a seed is the first output for the seed
+    advanced by j increments, so it pins every draw the hash routing takes."""
+    rnd = pytest.importorskip("numba.cuda.random")
+    st = np.zeros(1, dtype=rnd.xoroshiro128p_dtype)
+    gamma = 0x9E3779B97F4A7C15
+    for seed in (0, 1, 7, 12345, 129279, 2**32 + 3, 2**63 + 5):
+        ours = ora.splitmix64_outputs(seed, 4)
+        for j, o in enumerate(ours):
+            rnd.init_xoroshiro128p_state(st, 0, np.uint64((seed + j * gamma) % 2**64))
+            assert int(st[0]["s0"]) == o, (seed, j)
+
+
 def test_splitmix_outputs_distinct_and_uniform(ora):
     outs = ora.splitmix64_outputs(12345, 20000)
     assert len(set(outs)) == len(outs)
