@@ -191,6 +191,30 @@ def test_route_ties_to_lower_index():
     np.testing.assert_allclose(host(w), w_ref, atol=2e-6)
 
 
+@pytest.mark.parametrize("T", [8, 40])
+def test_route_nan_logits_rank_last(T):
+    """A token whose x row holds a NaN has NaN logits for every expert: they
+    all rank after every number and tie among themselves, so the token takes
+    experts 0 .. k-1 (and NaN gates); a token with one NaN-free logit row is
+    untouched. T = 40 runs the tiled router, T = 8 the per-token one."""
+    cfg = synth.LayerConfig("nan", T=T, d=256, F=256, E=16, k=4)
+    wr = synth.make_router(cfg)
+    x = synth.make_x(cfg)
+    x[1, 7] = 0x7FC0                      # bf16 quiet NaN
+    logits = oracle.router_logits(x, wr)
+    assert np.all(np.isnan(logits[1])) and not np.any(np.isnan(np.delete(logits, 1, axis=0)))
+    idx_ref, w_ref = oracle.topk_softmax(logits, cfg.k)
+    assert list(idx_ref[1]) == [0, 1, 2, 3]
+    dims = M.make_dims(cfg.T, cfg.d, cfg.F, cfg.E, cfg.k)
+    ws = torch.empty(M.moe_workspace_size(dims), dtype=torch.uint8, device=DEV)
+    weights = M.make_weights(None, None, None, w_router=dev(wr))
+    idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=DEV)
+    w = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=DEV)
+    M.moe_route(dims, dev(x), weights, None, idx, w, ws)
+    np.testing.assert_array_equal(host(idx), idx_ref)
+    np.testing.assert_allclose(host(w), w_ref, atol=2e-6)   # NaN gates compare equal
+
+
 @pytest.mark.parametrize("name,T", ROUTE_CASES)
 def test_permute_bitexact(name, T):
     c = get_case(name, T)
