@@ -176,6 +176,17 @@ def decode_traffic(cfg, T):
     return rec["dram_bytes"] if h.hexdigest() == rec["sources_sha256"] else None
 
 
+def hbm_fraction(M, torch, layer, cfg, T, r, hbm, rank):
+    """The decode roofline of one breakdown entry, as for the headline line:
+    experts touched by batch 0's routing, its algorithmic bytes over the mean
+    FFN time of the batch-0 steps, as a fraction of the HBM peak."""
+    xb = torch.from_numpy(synth.make_x(cfg, 0, 1000 * rank).astype(np.int16)).cuda()
+    U = len(np.unique(touched_experts(M, torch, layer, xb, None, T)))
+    f0 = statistics.mean(r["ffn_ms"][::NBATCH])
+    gbs = algorithmic_ffn_bytes(cfg, U) / (f0 / 1000.0) / 1e9
+    return {"experts_touched": U, "ffn_hbm_gbs": gbs, "ffn_hbm_frac": gbs / hbm}
+
+
 def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=False):
     """Times `steps` moe_layer calls; returns a dict of per-step times (ms)."""
     cfg = layer.cfg
@@ -498,9 +509,11 @@ def main():
         if cfg.wfmt == "mxfp4" and cfg.d == synth.CONFIGS["decode"].d:
             dec = replace(synth.CONFIGS["decode"], E=E)
             for Tb in (1, 2, 4, 8):
-                rr = measure(M, torch, base.with_weights(dec.with_T(Tb)), Tb, 20, 3, rank, 1)
+                lb = base.with_weights(dec.with_T(Tb))
+                rr = measure(M, torch, lb, Tb, 20, 3, rank, 1)
                 bd[f"decode_T{Tb}"] = {"tokens_per_s": Tb / (statistics.mean(rr["ms"]) / 1000),
-                                       "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
+                                       "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"]),
+                                       **hbm_fraction(M, torch, lb, dec.with_T(Tb), Tb, rr, hbm, rank)}
             for name in ("prefill", "hash"):
                 c = replace(synth.CONFIGS[name], E=E)
                 rr = measure(M, torch, base.with_weights(c), c.T, 3, 3, rank, 1, batches=2)
@@ -512,10 +525,12 @@ def main():
             torch.cuda.empty_cache()
             q2 = DeviceLayer(M, torch, replace(synth.CONFIGS["q2k"], E=E))
             for Tb in (1, 8):
-                rr = measure(M, torch, q2.with_weights(replace(synth.CONFIGS["q2k"], E=E).with_T(Tb)), Tb, 20, 3,
-                             rank, 1)
+                qc = replace(synth.CONFIGS["q2k"], E=E).with_T(Tb)
+                lb = q2.with_weights(qc)
+                rr = measure(M, torch, lb, Tb, 20, 3, rank, 1)
                 bd[f"q2k_T{Tb}"] = {"tokens_per_s": Tb / (statistics.mean(rr["ms"]) / 1000),
-                                    "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"])}
+                                    "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"]),
+                                    **hbm_fraction(M, torch, lb, qc, Tb, rr, hbm, rank)}
         line["breakdown"] = bd
 
     if not args.no_cpu and world == 1 and rank == 0:
