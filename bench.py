@@ -10,11 +10,14 @@ timed events. Other configurations are measured in the same run and reported
 under "breakdown".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config decode|prefill|hash|q2k|tiny] [--T T] [--E E]
+                    [--config decode|prefill|hash|q2k|tiny] [--T T] [--E E] [--ep]
 
 With N > 1 (torchrun) every rank runs an independent replica on its own
 batches (the path partitions by token batch; no data-path collective) and the
-job value is the sum over ranks of tokens over the slowest rank's time.
+job value is the sum over ranks of tokens over the slowest rank's time. With
+--ep the N ranks instead split one layer's routed experts (moe_layer_ep on a
+contiguous share each, the shared expert on rank 0, NCCL all-reduce of y):
+one batch per step, strong scaling.
 --impl reference times the oracle (plain C, host cores) on the same workload.
 """
 from __future__ import annotations
@@ -61,10 +64,15 @@ class DeviceLayer:
     """Weights of one layer config on the device, built with the library's own
     quantiser and packer from the seeded generator's fp32 normals."""
 
-    def __init__(self, M, torch, cfg, seed=0):
+    def __init__(self, M, torch, cfg, seed=0, experts=None):
+        """experts: (begin, end) to hold only those routed experts (one rank of
+        the expert-parallel layer); default all."""
         self.M, self.torch, self.cfg = M, torch, cfg
         dev = torch.device("cuda")
         self.dims = self.dims_for(cfg.T)
+        self.ebegin, self.eend = experts if experts else (0, cfg.E)
+        nE = self.eend - self.ebegin
+        local = M.make_dims(cfg.T, cfg.d, cfg.F, nE, cfg.k, self.dims.route, self.dims.act, self.dims.wfmt, 0)
         self.packed = {}
         chunk = 16
         for tid, which in ((synth.W1, M.MOE_MAT_W1), (synth.W3, M.MOE_MAT_W3), (synth.W2, M.MOE_MAT_W2)):
@@ -72,22 +80,23 @@ class DeviceLayer:
             q2k = cfg.wfmt == "q2k"
             per_e_a = N * K // 256 * 84 if q2k else N * K // 2
             per_e_b = 0 if q2k else N * K // 32
-            canon = torch.empty(cfg.E * (per_e_a + per_e_b), dtype=torch.uint8, device=dev)
+            canon = torch.empty(nE * (per_e_a + per_e_b), dtype=torch.uint8, device=dev)
             f32 = torch.empty(chunk * N * K, dtype=torch.float32, device=dev)
             tmp = torch.empty(chunk * (per_e_a + per_e_b), dtype=torch.uint8, device=dev)
-            for e0 in range(0, cfg.E, chunk):
-                ne = min(chunk, cfg.E - e0)
-                for j in range(ne):
-                    synth.normal_f32_device(seed, tid, e0 + j, N * K, 0.0, cfg.w_std, out=f32[j * N * K:(j + 1) * N * K])
+            for e0 in range(0, nE, chunk):
+                ne = min(chunk, nE - e0)
+                for j in range(ne):  # expert ids are the layer's: a rank's experts draw the same weights
+                    synth.normal_f32_device(seed, tid, self.ebegin + e0 + j, N * K, 0.0, cfg.w_std,
+                                            out=f32[j * N * K:(j + 1) * N * K])
                 cd = M.make_dims(1, cfg.d, cfg.F, ne, 1, wfmt=self.dims.wfmt)
                 M.moe_quantize_weights(cd, which, f32, tmp)
                 canon[e0 * per_e_a:(e0 + ne) * per_e_a].copy_(tmp[:ne * per_e_a])
                 if per_e_b:
-                    base = cfg.E * per_e_a
+                    base = nE * per_e_a
                     canon[base + e0 * per_e_b: base + (e0 + ne) * per_e_b].copy_(
                         tmp[ne * per_e_a: ne * (per_e_a + per_e_b)])
-            out = torch.empty(M.moe_packed_size(self.dims, which), dtype=torch.uint8, device=dev)
-            M.moe_pack_weights(self.dims, which, canon, out)
+            out = torch.empty(M.moe_packed_size(local, which), dtype=torch.uint8, device=dev)
+            M.moe_pack_weights(local, which, canon, out)
             self.packed[which] = out
             del canon, f32, tmp
         to16 = lambda a: torch.from_numpy(a.astype(np.int16)).to(dev)
@@ -187,17 +196,20 @@ def hbm_fraction(M, torch, layer, cfg, T, r, hbm, rank):
     return {"experts_touched": U, "ffn_hbm_gbs": gbs, "ffn_hbm_frac": gbs / hbm}
 
 
-def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=False):
-    """Times `steps` moe_layer calls; returns a dict of per-step times (ms)."""
+def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=False, ep=False):
+    """Times `steps` moe_layer calls; returns a dict of per-step times (ms).
+    ep: every rank runs its share of one expert-parallel layer on the same
+    batch (moe_layer_ep on its experts, then the all-reduce of y)."""
     cfg = layer.cfg
     dev = torch.device("cuda")
     dims = layer.dims_for(T)
     ws = torch.empty(M.moe_workspace_size(dims), dtype=torch.uint8, device=dev)
     xs, toks = [], []
+    src_rank = 0 if ep else rank  # expert parallelism: one batch, replicated on every rank
     for b in range(batches):
         c = cfg.with_T(T)
-        xs.append(torch.from_numpy(synth.make_x(c, 0, batch_index(rank, b)).astype(np.int16)).to(dev))
-        toks.append(torch.from_numpy(synth.make_token_ids(c, 0, batch_index(rank, b))).to(dev)
+        xs.append(torch.from_numpy(synth.make_x(c, 0, batch_index(src_rank, b)).astype(np.int16)).to(dev))
+        toks.append(torch.from_numpy(synth.make_token_ids(c, 0, batch_index(src_rank, b))).to(dev)
                     if cfg.route == "hash" else None)
     y = torch.empty((T, cfg.d), dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -216,6 +228,14 @@ def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=
         a.record(stream)
         b.record(stream)
 
+    def layer_call(x, tok):
+        if ep:
+            M.moe_layer_ep(dims, layer.weights, layer.ebegin, layer.eend, rank == 0, x, tok, y, ws)
+            if world > 1:
+                torch.distributed.all_reduce(y)
+        else:
+            M.moe_layer(dims, layer.weights, x, tok, y, ws)
+
     def step(i, timed, ffn_events=False):
         b = i % batches
         flush.fill_(i & 0xFF)
@@ -227,10 +247,10 @@ def measure(M, torch, layer, T, steps, warmup, rank, world, batches=NBATCH, e2e=
             xd.copy_(xh[b], non_blocking=True)
             if td is not None:
                 td.copy_(th[b], non_blocking=True)
-            M.moe_layer(dims, layer.weights, xd, td, y, ws)
+            layer_call(xd, td)
             yh.copy_(y, non_blocking=True)
         else:
-            M.moe_layer(dims, layer.weights, xs[b], toks[b], y, ws)
+            layer_call(xs[b], toks[b])
         if timed:
             if ffn_events:
                 M.moe_debug_set_ffn_events(None, None)
@@ -400,6 +420,9 @@ def main():
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: the N ranks split one layer's routed experts (one batch, "
+                         "partial sums all-reduced) instead of running N replicas")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -443,23 +466,27 @@ def main():
     import routed_expert_ffn_05_b200 as M
 
     t0 = time.time()
+    ep = args.ep
+    span = M.moe_ep_range(E, rank, world) if ep else None
     if cfg.wfmt == "q2k" or cfg.d != synth.CONFIGS["decode"].d:
-        base = DeviceLayer(M, torch, cfg)
+        base = DeviceLayer(M, torch, cfg, experts=span)
     else:
-        base = DeviceLayer(M, torch, replace(synth.CONFIGS["decode"], E=E))
+        base = DeviceLayer(M, torch, replace(synth.CONFIGS["decode"], E=E), experts=span)
     log(f"[bench] {cfg.wfmt} layer built in {time.time() - t0:.1f}s")
     layer = base.with_weights(cfg)
+    # replicas: every rank's tokens count; expert parallelism: the ranks share one batch
+    job_ranks = 1 if ep else world
 
     clocks = Clocks()
     clocks.start()
-    r = measure(M, torch, layer, T, args.steps, args.warmup, rank, world)
+    r = measure(M, torch, layer, T, args.steps, args.warmup, rank, world, ep=ep)
     ck = clocks.stop()
     total_s = max_over_ranks(torch, world, sum(r["ms"]) / 1000.0)
-    value = job_value(world, T, args.steps, total_s)
+    value = job_value(job_ranks, T, args.steps, total_s)
     ms_per_step = 1000.0 * total_s / args.steps
 
     if not args.no_e2e:
-        e = measure(M, torch, layer, T, args.steps, args.warmup, rank, world, e2e=True)
+        e = measure(M, torch, layer, T, args.steps, args.warmup, rank, world, e2e=True, ep=ep)
         e2e_s = max_over_ranks(torch, world, sum(e["ms"]) / 1000.0)
     else:
         e2e_s = float("nan")
@@ -476,11 +503,13 @@ def main():
                 "frac": achieved / peak, "peak_source": f"{src} bf16 x 2 (FP8 nominal ratio)",
                 "traffic": None, "algorithmic_flops": fl, "ffn_ms": ffn_ms}
     else:
-        xb = torch.from_numpy(synth.make_x(cfg, 0, 1000 * rank).astype(np.int16)).cuda()
+        xb = torch.from_numpy(synth.make_x(cfg, 0, 1000 * (0 if ep else rank)).astype(np.int16)).cuda()
         idx = touched_experts(M, torch, layer, xb, None, T)
+        if ep:  # this rank's experts (and the shared expert on rank 0 only)
+            idx = idx[(idx >= layer.ebegin) & (idx < layer.eend)]
         U = len(np.unique(idx))
         ffn_ms = statistics.mean(r["ffn_ms"][::NBATCH]) if r["ffn_ms"] else float("nan")
-        alg = algorithmic_ffn_bytes(cfg, U)
+        alg = algorithmic_ffn_bytes(cfg if not ep or rank == 0 else replace(cfg, Fs=0), U)
         achieved = alg / (ffn_ms / 1000.0) / 1e9
         roof = {"kernel": "expert FFN: routed + shared", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
@@ -488,23 +517,26 @@ def main():
                 "algorithmic_bytes": alg, "experts_touched": U, "ffn_ms": ffn_ms}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if ep else "weak",
         "vs_baseline": None,
         "dtype": ("mxfp4 x mxfp8 -> fp32" if cfg.act == "mxfp8" else
                   ("q2k x bf16 -> fp32" if cfg.wfmt == "q2k" else "mxfp4 x bf16 -> fp32")),
         "data": "synthetic",
         "config": {"workload": workload, "T": T, "batches": NBATCH,
                    "l2": "flushed between steps (256 MB write), flush outside the timed events",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": (f"expert-parallel x{world} (experts {layer.ebegin}..{layer.eend - 1} on rank 0, "
+                                   f"NCCL all-reduce of y)" if ep else
+                                   f"replicas x{world}" if world > 1 else "single GPU")},
         "roofline": roof,
-        "e2e": {"value": job_value(world, T, args.steps, e2e_s), "unit": UNIT,
+        "e2e": {"value": job_value(job_ranks, T, args.steps, e2e_s), "unit": UNIT,
                 "h2d_bytes_per_step": T * cfg.d * 2 + (T * 4 if cfg.route == "hash" else 0),
                 "d2h_bytes_per_step": T * cfg.d * 4},
         "gpu_launches": r["launches"], "gpu_launches_per_step": r["launches"] / args.steps,
         "clocks": ck,
     }
 
-    if not args.no_breakdown and rank == 0:
+    if not args.no_breakdown and rank == 0 and not ep:
         bd = {}
         if cfg.wfmt == "mxfp4" and cfg.d == synth.CONFIGS["decode"].d:
             dec = replace(synth.CONFIGS["decode"], E=E)

@@ -41,6 +41,10 @@ class moe_weights(ctypes.Structure):
                 ("w1", "w3", "w2", "sw1", "sw3", "sw2", "w_router", "router_bias")]
 
 
+class moe_cache_stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_uint64) for n in ("calls", "waves", "hits", "misses", "bytes_h2d")]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python routed_expert_ffn_05_b200/build.py`")
@@ -63,6 +67,16 @@ def _load():
         "moe_debug_dequant": (ctypes.c_int, [D, i32, vp, i32, vp, vp]),
         "moe_debug_quant_act": (ctypes.c_int, [vp, i32, i32, vp, vp, vp]),
         "moe_layer_static_ws": (ctypes.c_int, [D, W, vp, vp, vp, vp]),
+        "moe_ep_range": (ctypes.c_int, [i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]),
+        "moe_layer_ep": (ctypes.c_int, [D, W, i32, i32, i32, vp, vp, vp, vp, vp]),
+        "moe_cache_create": (ctypes.c_int, [D, i32, vp, vp, vp, vp, vp, vp, ctypes.POINTER(vp)]),
+        "moe_cache_destroy": (ctypes.c_int, [vp]),
+        "moe_cache_get_stats": (ctypes.c_int, [vp, ctypes.POINTER(moe_cache_stats)]),
+        "moe_layer_cached": (ctypes.c_int, [vp, D, W, vp, vp, vp, vp, vp]),
+        "moe_debug_hash_route": (ctypes.c_int, [D, vp, i32, vp, vp, vp]),
+        "moe_debug_tc_gather": (ctypes.c_int, [D, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "moe_debug_set_wait": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_uint32]),
+        "moe_debug_router_approx": (ctypes.c_int, [D, vp, W, vp, vp, vp]),
         "moe_debug_launch_count": (ctypes.c_uint64, []),
         "moe_debug_set_ffn_events": (ctypes.c_int, [vp, vp]),
     }
@@ -167,7 +181,79 @@ def moe_layer(dims, weights, x, token_ids, y, ws, stream=None):
                          _stream(stream)), "moe_layer")
 
 
-MOE_STATIC_WS_BYTES = 16 << 20
+def moe_ep_range(E, rank, world):
+    """(begin, end): the contiguous routed experts rank `rank` of `world` owns."""
+    b, e = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib.moe_ep_range(E, rank, world, ctypes.byref(b), ctypes.byref(e)), "moe_ep_range")
+    return b.value, e.value
+
+
+def moe_layer_ep(dims, weights, expert_begin, expert_end, add_shared, x, token_ids, y, ws, stream=None):
+    _check(lib.moe_layer_ep(ctypes.byref(dims), ctypes.byref(weights), expert_begin, expert_end, int(add_shared),
+                            _p(x), _p(token_ids), _p(y), _p(ws), _stream(stream)), "moe_layer_ep")
+
+
+def moe_layer_ep_allreduce(dims, weights, rank, world, x, token_ids, y, ws, group=None, stream=None):
+    """One rank of the expert-parallel layer: this rank's part (its experts,
+    plus the shared expert on rank 0) into y, then the sum over ranks in place
+    (torch.distributed all-reduce; NCCL on GPUs). Every rank ends with the
+    whole layer's y. ``weights`` holds this rank's experts (moe_ep_range)."""
+    import torch.distributed as dist
+    b, e = moe_ep_range(dims.E, rank, world)
+    moe_layer_ep(dims, weights, b, e, rank == 0, x, token_ids, y, ws, stream)
+    dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
+    return y
+
+
+class ExpertCache:
+    """moe_cache_create / moe_layer_cached / moe_cache_destroy: ``slots`` routed
+    experts in HBM (dev_w1/3/2), all of them in pinned host memory (host_w1/3/2,
+    packed layout). Keeps the buffers it was given alive."""
+
+    def __init__(self, dims, slots, host_w1, host_w3, host_w2, dev_w1, dev_w3, dev_w2):
+        self.handle = None
+        self._keep = (host_w1, host_w3, host_w2, dev_w1, dev_w3, dev_w2)
+        self.dims = dims
+        h = ctypes.c_void_p()
+        _check(lib.moe_cache_create(ctypes.byref(dims), slots, _p(host_w1), _p(host_w3), _p(host_w2), _p(dev_w1),
+                                    _p(dev_w3), _p(dev_w2), ctypes.byref(h)), "moe_cache_create")
+        self.handle = h.value
+
+    def layer(self, dims, weights, x, token_ids, y, ws, stream=None):
+        _check(lib.moe_layer_cached(self.handle, ctypes.byref(dims), ctypes.byref(weights), _p(x), _p(token_ids),
+                                    _p(y), _p(ws), _stream(stream)), "moe_layer_cached")
+
+    def stats(self) -> dict:
+        st = moe_cache_stats()
+        _check(lib.moe_cache_get_stats(self.handle, ctypes.byref(st)), "moe_cache_get_stats")
+        return {n: getattr(st, n) for n, _ in st._fields_}
+
+    def close(self):
+        if self.handle:
+            lib.moe_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        self.close()
+
+
+def moe_cache_create(dims, slots, host_w1, host_w3, host_w2, dev_w1, dev_w3, dev_w2) -> ExpertCache:
+    return ExpertCache(dims, slots, host_w1, host_w3, host_w2, dev_w1, dev_w3, dev_w2)
+
+
+def moe_cache_destroy(cache: ExpertCache):
+    cache.close()
+
+
+def moe_cache_get_stats(cache: ExpertCache) -> dict:
+    return cache.stats()
+
+
+def moe_layer_cached(cache: ExpertCache, dims, weights, x, token_ids, y, ws, stream=None):
+    cache.layer(dims, weights, x, token_ids, y, ws, stream)
+
+
+MOE_STATIC_WS_BYTES = 32 << 20
 
 
 def moe_layer_static_ws(dims, weights, x, token_ids, y, stream=None):
@@ -193,6 +279,25 @@ def moe_debug_dequant(dims, which, packed, expert, out, stream=None):
 def moe_debug_quant_act(x, rows, K, codes, scales, stream=None):
     _check(lib.moe_debug_quant_act(_p(x), rows, K, _p(codes), _p(scales), _stream(stream)),
            "moe_debug_quant_act")
+
+
+def moe_debug_hash_route(dims, token_ids, max_draws, topk_idx, topk_w, stream=None):
+    _check(lib.moe_debug_hash_route(ctypes.byref(dims), _p(token_ids), max_draws, _p(topk_idx), _p(topk_w),
+                                    _stream(stream)), "moe_debug_hash_route")
+
+
+def moe_debug_tc_gather(dims, x, offsets, perm, codes, atoms, ustart, ws, stream=None):
+    _check(lib.moe_debug_tc_gather(ctypes.byref(dims), _p(x), _p(offsets), _p(perm), _p(codes), _p(atoms),
+                                   _p(ustart), _p(ws), _stream(stream)), "moe_debug_tc_gather")
+
+
+def moe_debug_router_approx(dims, x, weights, approx, wnorm, stream=None):
+    _check(lib.moe_debug_router_approx(ctypes.byref(dims), _p(x), ctypes.byref(weights), _p(approx), _p(wnorm),
+                                       _stream(stream)), "moe_debug_router_approx")
+
+
+def moe_debug_set_wait(limit_ns=0, extra_tiles=0):
+    _check(lib.moe_debug_set_wait(limit_ns, extra_tiles), "moe_debug_set_wait")
 
 
 def moe_debug_launch_count() -> int:

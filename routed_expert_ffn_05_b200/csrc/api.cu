@@ -11,13 +11,18 @@ namespace moe {
 
 __device__ int g_device_error = 0;
 
+// Looked up once per device and kept for the life of the process (a
+// cudaDeviceReset would invalidate it; the library is not meant to outlive one).
 int *device_error_word() {
-    static int *addr[64] = {nullptr};
+    static std::atomic<int *> addr[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev] && cudaGetSymbolAddress(reinterpret_cast<void **>(&addr[dev]), g_device_error) != cudaSuccess)
-        return nullptr;
-    return addr[dev];
+    int *p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_device_error) != cudaSuccess) return nullptr;
+        addr[dev].store(p, std::memory_order_release);
+    }
+    return p;
 }
 
 static std::atomic<uint64_t> g_launches{0};
@@ -146,7 +151,8 @@ moe_status moe_route(const moe_dims *dims, const uint16_t *x, const moe_weights 
     if (dims->T > 0 && dims->route == MOE_ROUTE_SOFTMAX_TOPK && (!x || !aligned(x, 16))) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(*dims);
     float *logits = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.logits);
-    return cuda_status(launch_route(*dims, x, *weights, token_ids, topk_idx, topk_w, logits,
+    float *rnorm = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + L.rnorm);
+    return cuda_status(launch_route(*dims, x, *weights, token_ids, topk_idx, topk_w, logits, rnorm,
                                     static_cast<cudaStream_t>(stream)));
 }
 
@@ -202,6 +208,47 @@ moe_status moe_combine(const moe_dims *dims, const float *out_rows, const int32_
                                       static_cast<cudaStream_t>(stream)));
 }
 
+// The layer over the routed experts [ebase, ebase + El) of a layer of d.E
+// (all of them for moe_layer), plus the shared expert when add_shared. Routing
+// always runs over all d.E experts; the slots of experts outside the range
+// take no row and add nothing to y. `w` holds the El experts' routed weights.
+static moe_status layer_impl(const moe_dims &d, const moe_weights &wt, int ebase, int El, bool add_shared,
+                             const uint16_t *x, const int32_t *token_ids, float *y, void *ws, cudaStream_t s) {
+    const WsLayout L = ws_layout(d);  // the whole layer's layout covers every sub-range
+    moe_dims dl = d;                  // the experts (and shared expert) this call computes
+    dl.E = El;
+    if (!add_shared) dl.d_ff_shared = 0;
+    const bool part = El != d.E;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    int32_t *idx = reinterpret_cast<int32_t *>(w + L.topk_idx);
+    float *gates = reinterpret_cast<float *>(w + L.topk_w);
+    int32_t *counts = reinterpret_cast<int32_t *>(w + L.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
+    int32_t *perm = reinterpret_cast<int32_t *>(w + L.perm);
+    int32_t *inv = reinterpret_cast<int32_t *>(w + L.inv_perm);
+    float *rows = reinterpret_cast<float *>(w + L.out_rows);
+    float *sh = dl.d_ff_shared > 0 ? reinterpret_cast<float *>(w + L.sh_out) : nullptr;
+    cudaError_t e;
+    const bool fused = decode_route_applies(d) && decode_path_applies(dl);
+    if (fused) {
+        if ((e = launch_decode_route(d, x, wt, idx, gates, counts, offsets, perm, inv, w, L, s, ebase, El)))
+            return cuda_status(e);
+    } else {
+        if ((e = launch_route(d, x, wt, token_ids, idx, gates, reinterpret_cast<float *>(w + L.logits),
+                              reinterpret_cast<float *>(w + L.rnorm), s)))
+            return cuda_status(e);
+        if ((e = launch_permute(dl, idx, counts, offsets, perm, inv, reinterpret_cast<int32_t *>(w + L.blkcnt),
+                                reinterpret_cast<int32_t *>(w + L.blkbase), L.nblk, s, ebase, part)))
+            return cuda_status(e);
+    }
+    // the tensor-core path hands its rows to the combine as bf16 (half the traffic)
+    const bool r16 = tc_path_applies(dl);
+    if ((e = expert_ffn_timed(dl, wt, x, offsets, perm, rows, sh, w, L, s, fused, r16))) return cuda_status(e);
+    if (r16)
+        return cuda_status(launch_combine_bf16(dl, reinterpret_cast<const uint16_t *>(rows), inv, gates, sh, y, s));
+    return cuda_status(launch_combine(dl, rows, inv, gates, sh, y, s, decode_path_applies(dl)));
+}
+
 moe_status moe_layer(const moe_dims *dims, const moe_weights *weights, const uint16_t *x,
                      const int32_t *token_ids, float *y, void *ws, void *stream) {
     moe_status st = check_dims(dims);
@@ -211,36 +258,33 @@ moe_status moe_layer(const moe_dims *dims, const moe_weights *weights, const uin
     if (dims->T > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return MOE_ERR_INVALID_ARG;
     if (dims->T > 0 && dims->route == MOE_ROUTE_HASH && !token_ids) return MOE_ERR_INVALID_ARG;
     if (dims->T == 0) return MOE_OK;
-    const moe_dims &d = *dims;
-    const WsLayout L = ws_layout(d);
-    uint8_t *w = static_cast<uint8_t *>(ws);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    int32_t *idx = reinterpret_cast<int32_t *>(w + L.topk_idx);
-    float *gates = reinterpret_cast<float *>(w + L.topk_w);
-    int32_t *counts = reinterpret_cast<int32_t *>(w + L.counts);
-    int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
-    int32_t *perm = reinterpret_cast<int32_t *>(w + L.perm);
-    int32_t *inv = reinterpret_cast<int32_t *>(w + L.inv_perm);
-    float *rows = reinterpret_cast<float *>(w + L.out_rows);
-    float *sh = d.d_ff_shared > 0 ? reinterpret_cast<float *>(w + L.sh_out) : nullptr;
-    cudaError_t e;
-    const bool fused = decode_route_applies(d);
-    if (fused) {
-        if ((e = launch_decode_route(d, x, *weights, idx, gates, counts, offsets, perm, inv, w, L, s)))
-            return cuda_status(e);
-    } else {
-        if ((e = launch_route(d, x, *weights, token_ids, idx, gates, reinterpret_cast<float *>(w + L.logits), s)))
-            return cuda_status(e);
-        if ((e = launch_permute(d, idx, counts, offsets, perm, inv, reinterpret_cast<int32_t *>(w + L.blkcnt),
-                                reinterpret_cast<int32_t *>(w + L.blkbase), L.nblk, s)))
-            return cuda_status(e);
-    }
-    // the tensor-core path hands its rows to the combine as bf16 (half the traffic)
-    const bool r16 = tc_path_applies(d);
-    if ((e = expert_ffn_timed(d, *weights, x, offsets, perm, rows, sh, w, L, s, fused, r16))) return cuda_status(e);
-    if (r16)
-        return cuda_status(launch_combine_bf16(d, reinterpret_cast<const uint16_t *>(rows), inv, gates, sh, y, s));
-    return cuda_status(launch_combine(d, rows, inv, gates, sh, y, s, decode_path_applies(d)));
+    return layer_impl(*dims, *weights, 0, dims->E, true, x, token_ids, y, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_ep_range(int32_t E, int32_t rank, int32_t world, int32_t *begin, int32_t *end) {
+    if (E <= 0 || world <= 0 || world > E || rank < 0 || rank >= world || !begin || !end) return MOE_ERR_INVALID_ARG;
+    *begin = (int32_t)((int64_t)E * rank / world);
+    *end = (int32_t)((int64_t)E * (rank + 1) / world);
+    return MOE_OK;
+}
+
+moe_status moe_layer_ep(const moe_dims *dims, const moe_weights *weights, int32_t expert_begin, int32_t expert_end,
+                        int32_t add_shared, const uint16_t *x, const int32_t *token_ids, float *y, void *ws,
+                        void *stream) {
+    moe_status st = check_dims(dims);
+    if (st != MOE_OK) return st;
+    if (expert_begin < 0 || expert_end <= expert_begin || expert_end > dims->E) return MOE_ERR_INVALID_ARG;
+    moe_dims dw = *dims;  // the weights' own shape: expert_end - expert_begin routed experts
+    dw.E = expert_end - expert_begin;
+    if (!add_shared) dw.d_ff_shared = 0;
+    if ((st = check_weights(&dw, weights, true, false, true)) != MOE_OK) return st;
+    if ((st = check_weights(dims, weights, false, true, false)) != MOE_OK) return st;
+    if ((st = check_ws(dims, ws)) != MOE_OK) return st;
+    if (dims->T > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return MOE_ERR_INVALID_ARG;
+    if (dims->T > 0 && dims->route == MOE_ROUTE_HASH && !token_ids) return MOE_ERR_INVALID_ARG;
+    if (dims->T == 0) return MOE_OK;
+    return layer_impl(*dims, *weights, expert_begin, expert_end - expert_begin, add_shared != 0, x, token_ids, y, ws,
+                      static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_get_device_error(void *stream, int32_t *code) {
@@ -271,6 +315,43 @@ moe_status moe_debug_quant_act(const uint16_t *x, int32_t rows, int32_t K, uint8
     if (rows < 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
     if (rows > 0 && (!x || !codes || !scales || !aligned(codes, 16))) return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_quant_act_bf16(x, rows, K, codes, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_debug_hash_route(const moe_dims *dims, const int32_t *token_ids, int32_t max_draws, int32_t *topk_idx,
+                                float *topk_w, void *stream) {
+    moe_status st = check_dims(dims);
+    if (st != MOE_OK) return st;
+    if (dims->route != MOE_ROUTE_HASH || max_draws < 1 || max_draws > kHashMaxDraws) return MOE_ERR_INVALID_ARG;
+    if (dims->T > 0 && (!token_ids || !topk_idx || !topk_w)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_hash_route(*dims, token_ids, max_draws, topk_idx, topk_w, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_debug_tc_gather(const moe_dims *dims, const uint16_t *x, const int32_t *offsets, const int32_t *perm,
+                               uint8_t *codes, uint8_t *atoms, int32_t *ustart, void *ws, void *stream) {
+    moe_status st = check_dims(dims);
+    if (st != MOE_OK) return st;
+    if (!tc_path_applies(*dims)) return MOE_ERR_UNSUPPORTED;
+    if ((st = check_ws(dims, ws)) != MOE_OK) return st;
+    if (!x || !offsets || !perm || !codes || !atoms || !ustart || !aligned(x, 16) || !aligned(codes, 16))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*dims);
+    return cuda_status(launch_tc_gather(*dims, x, offsets, perm, ustart,
+                                       reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + L.row_of), codes,
+                                       atoms, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_debug_router_approx(const moe_dims *dims, const uint16_t *x, const moe_weights *weights,
+                                  float *approx, float *wnorm, void *stream) {
+    moe_status st = check_dims(dims);
+    if (st != MOE_OK) return st;
+    if ((st = check_weights(dims, weights, false, true, false)) != MOE_OK) return st;
+    if (!router_tc_applies(*dims)) return MOE_ERR_UNSUPPORTED;
+    if (!x || !approx || !wnorm || !aligned(x, 16)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_router_approx(*dims, x, *weights, approx, wnorm, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_debug_set_wait(uint64_t limit_ns, uint32_t extra_tiles) {
+    return cuda_status(set_debug_wait(limit_ns, extra_tiles));
 }
 
 uint64_t moe_debug_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

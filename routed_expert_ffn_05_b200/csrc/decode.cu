@@ -14,10 +14,15 @@
 //    tiles (double-buffered) and writes the outputs;
 //  - the work is numbered in units (a unit: one or more stages the consumers
 //    run back to back, then one hand-off to the epilogue): shared gate/up
-//    (static per CTA, streamed while routing finishes), routed gate/up (a
-//    cost-balanced static range per CTA plus a dynamic tail from a queue),
-//    then down units as one contiguous static range per CTA; a down unit
-//    waits (bounded) on a per-expert count of finished gate/up tiles;
+//    (streamed while routing finishes), routed gate/up, then down units; a
+//    down unit waits (bounded) on a per-expert count of finished gate/up
+//    tiles. CTAs claim the work in chunks from one ticket counter, in unit
+//    order: shared gate/up units one at a time, routed gate/up as one large
+//    chunk per CTA's worth of three quarters of it and then pairs, down units
+//    as contiguous cost-balanced ranges. Every unit a down unit waits for was
+//    claimed earlier by a CTA that is running and finishes its earlier claims
+//    first, so the kernel needs no co-residency of its CTAs (other work may
+//    hold some SMs, or a second layer may run on another stream);
 //  - the producer stores each stage's decoded unit next to its data, so the
 //    consumers read one word instead of decoding unit numbers;
 //  - MXFP4 codes become f16 with the hardware E2M1 conversion; the E8M0 block
@@ -34,6 +39,8 @@
 // lane q of a quad holds elements 8q..8q+7 of a block, which cover its MMA
 // k-slots of both k16 steps.
 #include <string.h>
+
+#include <atomic>
 
 #include <cuda_fp16.h>
 
@@ -93,7 +100,8 @@ struct DecodeArgs {
     uint16_t *hs;            // shared hidden [T][Fs] bf16
     float *out_rows;         // [S][d]
     float *shared_out;       // [T][d]
-    uint32_t *counters;      // [0] work queue, [1] shared gate/up tiles done, [2+s] gate/up tiles done of active expert s
+    uint32_t *counters;      // [0] work ticket, [1] shared gate/up tiles done, [2+s] gate/up tiles done of active expert s
+                             // (all zeroed by a memset before the first kernel of the layer)
     int *err;
 };
 
@@ -186,15 +194,24 @@ __device__ __forceinline__ void fail(const DecodeArgs &a, S &s) {
     s.abort = 1;
 }
 
+// Test hooks for the inter-CTA wait below (moe_debug_set_wait): a shorter
+// limit, and extra tiles to wait for that no CTA ever publishes. Zero = off.
+__device__ uint64_t g_dbg_wait_ns = 0;
+__device__ uint32_t g_dbg_wait_extra = 0;
+
 // Bounded wait until *p >= target (another CTA's release). Lane 0 polls with
 // backoff; every lane then acquires for itself.
-__device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t target, int lane) {
+__device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t target, int lane, const volatile int *abort) {
     bool ok = true;
-    if (lane == 0 && ld_acquire(p) < target) {
-        const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire(p) < target) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) { ok = false; break; }
-            __nanosleep(256);
+    if (lane == 0) {
+        target += g_dbg_wait_extra;
+        if (ld_acquire(p) < target) {
+            const uint64_t lim = g_dbg_wait_ns ? g_dbg_wait_ns : kWaitLimitNs;
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire(p) < target) {
+                if (*abort || globaltimer_ns() - t0 > lim) { ok = false; break; }
+                __nanosleep(256);
+            }
         }
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -437,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             if (un.kind == kDrt) row0 = s.seg_e[un.seg] * kD + dn_rows<WF>() * un.tile;
             for (int c = 0; c < un.nst && !s.abort; ++c, ++gi) {
                 const int slot = gi % kStages;
-                if (!mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1)) { fail(a, s); return; }
+                if (!mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1, &s.abort)) { fail(a, s); return; }
                 uint8_t *w = s.w[slot];
                 uint8_t *sm = &s.s[0][0] + (size_t)slot * kStageS;  // the stage's scale / metadata bytes
                 uint64_t *bar = &s.full[slot];
@@ -482,10 +499,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 }
             }
         };
+        // Work tickets: [0, usg) are the shared gate/up units, one each; they
+        // need no routing, so they are claimed before the grid dependency
+        // resolves. The counter was zeroed before the routing kernels ran.
+        uint32_t *ticket = a.counters;
+        int t = 0;
         if (lane == 0) {
             prefetch_tensormap(&a.m1c);
             prefetch_tensormap(&a.m2c);
-            for (int u = blockIdx.x; u < usg && !s.abort; u += gridDim.x) issue(u, unit_of<WF>(u, usg, 0, 0));
+            t = (int)atomicAdd(ticket, 1u);
+            while (t < usg && !s.abort) {
+                const int nt = (int)atomicAdd(ticket, 1u);  // the next claim is fetched one chunk ahead
+                issue(t, unit_of<WF>(t, usg, 0, 0));
+                t = nt;
+            }
         }
         __syncwarp();
         grid_dep_wait();  // routing results and zeroed counters from here on
@@ -498,50 +525,60 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         }
         if (lane != 0) return;
         s.n_seg = n;
+        const int G = (int)gridDim.x;
         const int gu_end = usg + n * kGuTiles;
-        // Routed gate/up: the first three quarters as one static, stage-balanced
-        // range per CTA (no atomics; CTAs that carry a shared unit take 8 fewer
-        // stages), the last quarter from the queue in chunks of kGrab, which
-        // evens out CTAs that started late or ran slow. Falls back to the
-        // queue alone when the static split would not be monotonic.
-        const int R = n * kGuTiles;
-        int Rs = R - R / 4;
-        constexpr int kGuSt = gu_stages<WF>();
-        const long long tot = 8ll * usg + (long long)kGuSt * Rs;
-        if (usg > (int)gridDim.x || tot < 8ll * gridDim.x) Rs = 0;
-        auto rstart = [&](int b) {
-            const long long st = tot * b / gridDim.x - 8ll * min(b, usg);
-            return (int)min((long long)Rs, max(0ll, (st + kGuSt - 1) / kGuSt));
-        };
-        const int rs0 = Rs ? rstart(blockIdx.x) : 0, rs1 = Rs ? rstart(blockIdx.x + 1) : 0;
-        for (int u = usg + rs0; u < usg + rs1 && !s.abort; ++u) issue(u, unit_of<WF>(u, usg, n, usd));
+        // Routed gate/up tickets: G chunks of cb units that hold three quarters
+        // of the work (one per CTA when all run at once), then chunks of kGrab
+        // units, which even out CTAs that started late or ran slow.
         constexpr int kGrab = 2;
-        int next = usg + Rs + (int)atomicAdd(a.counters, (uint32_t)kGrab);
-        while (!s.abort) {  // the next chunk is fetched one chunk ahead
-            const int u0 = next;
-            if (u0 >= gu_end) break;
-            next = usg + Rs + (int)atomicAdd(a.counters, (uint32_t)kGrab);
-            for (int u = u0; u < min(u0 + kGrab, gu_end) && !s.abort; ++u) issue(u, unit_of<WF>(u, usg, n, usd));
-        }
-        // this CTA's contiguous share of the down units (shared tiles cost 2
-        // stages, routed ones dn_stages)
+        const int R = n * kGuTiles;
+        const int cb = (R - R / 4) / G;
+        const int nb = cb >= kGrab ? G : 0;
+        const int t_small = usg + nb, t_dn = t_small + (R - nb * cb + kGrab - 1) / kGrab;
+        // Down tickets: G contiguous ranges of equal cost (shared tiles cost 2
+        // stages, routed ones dn_stages), so a CTA changes expert, and reloads
+        // its h fragments, once or twice.
         constexpr int kDst = dn_stages<WF>();
         const long long cost = 2ll * usd + (long long)n * dn_tiles<WF>() * kDst;
         auto first = [&](long long cst) {
             return gu_end + (cst <= 2ll * usd ? (int)((cst + 1) / 2)
                                               : usd + (int)((cst - 2ll * usd + kDst - 1) / kDst));
         };
-        const int d0 = first(cost * blockIdx.x / gridDim.x), d1 = first(cost * (blockIdx.x + 1) / gridDim.x);
-        for (int u = d0; u < d1 && !s.abort; ++u) issue(u, unit_of<WF>(u, usg, n, usd));
+        const int t_end = t_dn + G;
+        while (t < t_end && !s.abort) {
+            int u0, u1;
+            if (t < usg) {
+                u0 = t;
+                u1 = t + 1;
+            } else if (t < t_small) {
+                u0 = usg + (t - usg) * cb;
+                u1 = u0 + cb;
+            } else if (t < t_dn) {
+                u0 = usg + nb * cb + (t - t_small) * kGrab;
+                u1 = min(u0 + kGrab, gu_end);
+            } else {
+                u0 = first(cost * (t - t_dn) / G);
+                u1 = first(cost * (t - t_dn + 1) / G);
+            }
+            // The next chunk is claimed while this chunk's last unit is issued
+            // (the ring keeps the consumers a few stages behind), not earlier:
+            // a CTA must not sit on a second large chunk while others idle.
+            int nt = -1;
+            for (int u = u0; u < u1 && !s.abort; ++u) {
+                if (u == u1 - 1) nt = (int)atomicAdd(ticket, 1u);
+                issue(u, unit_of<WF>(u, usg, n, usd));
+            }
+            t = nt >= 0 ? nt : (int)atomicAdd(ticket, 1u);
+        }
         if (!s.abort) {
             const int slot = gi % kStages;
-            if (mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1)) {
+            if (mbar_wait(&s.empty[slot], ((gi / kStages) & 1) ^ 1, &s.abort)) {
                 s.meta_u[slot] = -1;
                 mbar_arrive(&s.full[slot]);
+                ++gi;
             } else {
                 fail(a, s);
             }
-            ++gi;
         }
         for (int g = gi - kStages; g < gi; ++g)  // copies in flight finish before exit
             if (g >= 0) mbar_wait(&s.full[g % kStages], (g / kStages) & 1);
@@ -588,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         float dsc = 1.f;        // lane i < 8: output scale of row i of segment dseg
         for (int ru = 0;; ++ru) {
             const int rb = ru & 1;
-            if (!mbar_wait(&s.rfull[rb], (ru >> 1) & 1)) { fail(a, s); return; }
+            if (!mbar_wait(&s.rfull[rb], (ru >> 1) & 1, &s.abort)) { fail(a, s); return; }
             const int m = s.rmeta[rb];
             if (m == -1) return;
             if (m == -2) {  // before this CTA's first down unit: publish everything
@@ -707,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     auto code_off = [&](uint32_t base, int jj) { return base ^ ((uint32_t)jj << 4); };
     auto marker = [&](int m) {  // a hand-off without a tile: -1 end, -2 publish
         const int rb = ru & 1;
-        if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) return false;
+        if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1, &s.abort)) return false;
         if (threadIdx.x == 0) s.rmeta[rb] = m;
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.rfull[rb]);
@@ -728,10 +765,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     };
     auto next_stage = [&]() {  // the unit's next stage: wait until its data is in
         advance();
-        return mbar_wait(&s.full[slot], ph);
+        return mbar_wait(&s.full[slot], ph, &s.abort);
     };
     for (;; advance()) {
-        if (!mbar_wait(&s.full[slot], ph)) { fail(a, s); return; }
+        if (!mbar_wait(&s.full[slot], ph, &s.abort)) { fail(a, s); return; }
         const int u = s.meta_u[slot];
         if (u < 0) {  // end of work: publish (if still due) and tell the epilogue
             if ((!flushed && !marker(-2)) || !marker(-1)) fail(a, s);
@@ -752,8 +789,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     if (!marker(-2)) { fail(a, s); return; }
                     flushed = true;
                 }
-                const bool ok = un.kind == kDsh ? wait_count(sh_done, (uint32_t)usg, lane)
-                                                : wait_count(seg_done + un.seg, (uint32_t)kGuTiles, lane);
+                const bool ok = un.kind == kDsh ? wait_count(sh_done, (uint32_t)usg, lane, &s.abort)
+                                                : wait_count(seg_done + un.seg, (uint32_t)kGuTiles, lane, &s.abort);
                 if (!ok) { fail(a, s); return; }
             }
             if (Q2 && un.kind == kGrt) {  // x: super-block `warp` of K
@@ -864,7 +901,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             // dn_stages stages of 32 W2 rows over all K (rows 16 t + g (+ 8) of
             // each); B (the expert's h rows) is the same for all of them. The
             // partial tiles go out per stage, so the buffer is claimed first.
-            if (!mbar_wait(&s.rempty[ru & 1], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
+            if (!mbar_wait(&s.rempty[ru & 1], ((ru >> 1) & 1) ^ 1, &s.abort)) { fail(a, s); return; }
             float *red = s.red[ru & 1][warp];
 #pragma unroll
             for (int c = 0; c < dn_stages<WF>(); ++c) {
@@ -895,7 +932,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         // put their tiles in place already)
         const int rb = ru & 1;
         if (Q2 || un.kind != kDrt) {
-            if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1)) { fail(a, s); return; }
+            if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1, &s.abort)) { fail(a, s); return; }
             const int rg = (un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;  // bf16 tiles read rows sigma(g)
             put_partial(s.red[rb][warp], rg, q, acc[0]);
             if (un.kind != kDsh) put_partial(s.red[rb][warp] + kRedM, rg, q, acc[1]);
@@ -911,7 +948,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 // Decode routing: fixed-order fp32 logits (one CTA per expert, one warp per
 // token, lane = chunk; CTA 0 also computes the per-token f16 prescale), then
 // one CTA does top-k, softmax gates, histogram / scan / permutation and
-// resets the FFN kernel's scratch.
+// resets the FFN kernel's per-row h maxima.
 // ---------------------------------------------------------------------------
 // One CTA per expert, one warp per token: lane c runs the fma chain over
 // chunk c (elements 128 c .. 128 c + 127) in element order, then the fixed
@@ -971,10 +1008,11 @@ __global__ void __launch_bounds__(256) decode_logits_kernel(const uint16_t *__re
 
 struct FinalizeArgs {
     int T, E, k;
+    int ebase, El;  // this call's experts: ids [ebase, ebase + El) (the whole layer: 0, E)
     const float *logits;
     int32_t *idx, *counts, *offsets, *perm, *inv_perm;
     float *gates;
-    uint32_t *hmax, *counters;
+    uint32_t *hmax;
 };
 
 __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs a) {
@@ -985,7 +1023,6 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, E = a.E, k = a.k;
     grid_dep_launch();
-    for (int i = threadIdx.x; i < E + 2; i += blockDim.x) a.counters[i] = 0u;
     for (int i = threadIdx.x; i < T * k; i += blockDim.x) a.hmax[i] = 0u;
     grid_dep_wait();
     for (int base = 0; base < T * E; base += 8 * 256) {  // 8 loads in flight per thread
@@ -1001,7 +1038,7 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
             if (i < T * E) lg[i] = v[j];
         }
     }
-    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = run[e] = 0;
+    for (int e = threadIdx.x; e < a.El; e += blockDim.x) hist[e] = run[e] = 0;
     __syncthreads();
     if (warp < T) {  // top-k + gates of token `warp`: lane holds experts lane + 32 i
         const float *l = lg + warp * E;
@@ -1017,11 +1054,14 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
         }
     }
     __syncthreads();
-    const int S = T * k;
-    if (threadIdx.x < S) atomicAdd(&hist[sidx[threadIdx.x]], 1);
+    const int S = T * k, El = a.El;
+    if (threadIdx.x < S) {
+        const int e = sidx[threadIdx.x] - a.ebase;
+        if (e >= 0 && e < El) atomicAdd(&hist[e], 1);
+    }
     __syncthreads();
-    if (warp == 0) {  // exclusive scan over experts; lane owns experts [lane * per, (lane + 1) * per)
-        const int per = (E + 31) / 32, e0 = lane * per, e1 = min(E, e0 + per);
+    if (warp == 0) {  // exclusive scan over this call's experts; lane owns [lane * per, (lane + 1) * per)
+        const int per = (El + 31) / 32, e0 = lane * per, e1 = min(El, e0 + per);
         int tot = 0;
         for (int e = e0; e < e1; ++e) tot += hist[e];
         int incl = tot;
@@ -1038,7 +1078,7 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
             hist[e] = off;  // first row of expert e
             off += c;
         }
-        if (lane == 31) a.offsets[E] = incl;
+        if (lane == 31) a.offsets[El] = incl;
     }
     __syncthreads();
     // stable rank of each slot among the earlier slots of its expert: within a
@@ -1046,13 +1086,16 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
     for (int w0 = 0; w0 * 32 < S; ++w0) {
         if (warp == w0) {
             const int s0 = threadIdx.x;
-            const bool in = s0 < S;
-            const int e = in ? sidx[s0] : -1 - lane;
+            const int el = s0 < S ? sidx[s0] - a.ebase : -1;
+            const bool in = el >= 0 && el < El;  // a slot of another rank's expert gets no row
+            const int e = in ? el : -1 - lane;
             const unsigned peers = __match_any_sync(0xffffffffu, e);
             if (in) {
                 const int row = hist[e] + run[e] + __popc(peers & ((1u << lane) - 1u));
                 a.perm[row] = s0;
                 a.inv_perm[s0] = row;
+            } else if (s0 < S) {
+                a.inv_perm[s0] = -1;
             }
             __syncwarp();
             if (in && lane == 31 - __clz(peers)) run[e] += __popc(peers);
@@ -1061,9 +1104,9 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const FinalizeArgs
     }
 }
 
-// Stage-API entry (no routing in this call): the x prescale and the scratch reset.
-__global__ void __launch_bounds__(256) decode_prep_kernel(const uint16_t *__restrict__ x, int T, int S, int E,
-                                                          float2 *xscale, uint32_t *hmax, uint32_t *counters) {
+// Stage-API entry (no routing in this call): the x prescale and the h maxima reset.
+__global__ void __launch_bounds__(256) decode_prep_kernel(const uint16_t *__restrict__ x, int T, int S,
+                                                          float2 *xscale, uint32_t *hmax) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp < T) {
         float mx = 0.f;
@@ -1082,7 +1125,6 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(const uint16_t *__rest
         }
     }
     for (int i = threadIdx.x; i < S; i += blockDim.x) hmax[i] = 0u;
-    for (int i = threadIdx.x; i < E + 2; i += blockDim.x) counters[i] = 0u;
 }
 
 int num_sms() {
@@ -1092,10 +1134,10 @@ int num_sms() {
 }
 
 cudaError_t set_smem_attrs() {
-    static bool done[64] = {false};
+    static std::atomic<bool> done[64];  // per device; a repeated set-up from racing threads is harmless
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (done[dev]) return cudaSuccess;
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(decode_ffn_kernel<MOE_W_MXFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem_bytes<MOE_W_MXFP4>())))
@@ -1103,7 +1145,7 @@ cudaError_t set_smem_attrs() {
     if ((e = cudaFuncSetAttribute(decode_ffn_kernel<MOE_W_Q2K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem_bytes<MOE_W_Q2K>())))
         return e;
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
     return cudaSuccess;
 }
 
@@ -1127,6 +1169,12 @@ cudaError_t launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cuda
 
 }  // namespace
 
+cudaError_t set_debug_wait(uint64_t limit_ns, uint32_t extra) {
+    cudaError_t e = cudaMemcpyToSymbol(g_dbg_wait_ns, &limit_ns, sizeof limit_ns);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_dbg_wait_extra, &extra, sizeof extra);
+    return e;
+}
+
 bool decode_path_applies(const moe_dims &d) {
     // the tiling is written for d_model 4096, d_ff 2048 (and a shared d_ff of 2048)
     return d.T >= 1 && d.T <= 8 && (d.wfmt == MOE_W_MXFP4 || d.wfmt == MOE_W_Q2K) && d.act == MOE_A_BF16 &&
@@ -1142,17 +1190,22 @@ bool decode_route_applies(const moe_dims &d) {
 // reset for the FFN kernel). The logits kernel also writes the x prescale.
 cudaError_t launch_decode_route(const moe_dims &d, const uint16_t *x, const moe_weights &w, int32_t *idx,
                                 float *gates, int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm,
-                                uint8_t *ws, const WsLayout &L, cudaStream_t s) {
+                                uint8_t *ws, const WsLayout &L, cudaStream_t s, int ebase, int El) {
     cudaError_t e = set_smem_attrs();
     if (e != cudaSuccess) return e;
     float *logits = reinterpret_cast<float *>(ws + L.logits);
+    // the FFN kernel's work ticket and tile counts start at zero; the ticket is
+    // taken before the FFN kernel waits for these routing kernels, so it is
+    // reset here, ahead of them in stream order
+    if ((e = cudaMemsetAsync(ws + L.counters, 0, (size_t)(d.E + 2) * 4, s)) != cudaSuccess) return e;  // E >= El
     decode_logits_kernel<<<d.E, 32 * d.T, 0, s>>>(x, w.w_router, w.router_bias, d.T, d.E, logits,
                                                   reinterpret_cast<float2 *>(ws + L.xscale));
     FinalizeArgs f;
     f.T = d.T; f.E = d.E; f.k = d.k; f.logits = logits;
+    f.ebase = ebase;
+    f.El = El < 0 ? d.E : El;
     f.idx = idx; f.counts = counts; f.offsets = offsets; f.perm = perm; f.inv_perm = inv_perm; f.gates = gates;
     f.hmax = reinterpret_cast<uint32_t *>(ws + L.hmax);
-    f.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
     if ((e = launch_pdl(decode_finalize_kernel, dim3(1), dim3(256), 0, s, f)) != cudaSuccess) return e;
     count_launches(2);
     return cudaGetLastError();
@@ -1160,7 +1213,8 @@ cudaError_t launch_decode_route(const moe_dims &d, const uint16_t *x, const moe_
 
 // Routed + shared expert FFN for decode batches in one launch. `shared_out`
 // may be null. `prepared`: the decode routing already ran on this workspace
-// (x prescale, scratch reset); otherwise a small kernel does that first.
+// (x prescale, counters and h maxima reset); otherwise a memset and a small
+// kernel do that first.
 cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
                               const int32_t *perm, float *out_rows, float *shared_out, uint8_t *ws,
                               const WsLayout &L, cudaStream_t s, bool prepared) {
@@ -1210,8 +1264,8 @@ cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uin
     a.counters = reinterpret_cast<uint32_t *>(ws + L.counters);
     a.err = device_error_word();
     if (!prepared) {
-        decode_prep_kernel<<<1, 256, 0, s>>>(x, d.T, d.T * d.k, d.E, reinterpret_cast<float2 *>(ws + L.xscale), a.hmax,
-                                              a.counters);
+        if ((e = cudaMemsetAsync(a.counters, 0, (size_t)(d.E + 2) * 4, s)) != cudaSuccess) return e;
+        decode_prep_kernel<<<1, 256, 0, s>>>(x, d.T, d.T * d.k, reinterpret_cast<float2 *>(ws + L.xscale), a.hmax);
         count_launches(1);
     }
     e = q2 ? launch_pdl(decode_ffn_kernel<MOE_W_Q2K>, dim3(num_sms()), dim3(kThreads), smem_bytes<MOE_W_Q2K>(), s, a)

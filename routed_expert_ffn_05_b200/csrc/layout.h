@@ -74,9 +74,9 @@ static inline Q2kLayout q2k_layout(const moe_dims &d, int which) {
 
 // Workspace regions (byte offsets), one layout for every entry point.
 struct WsLayout {
-    int64_t logits, topk_idx, topk_w, counts, offsets, perm, inv_perm, blkcnt, blkbase;
+    int64_t logits, rnorm, topk_idx, topk_w, counts, offsets, perm, inv_perm, blkcnt, blkbase;
     int64_t x8, xs, xscale, counters, h, hmax, h8, hs, out_rows, sh_h, sh_out;
-    int64_t ustart, row_of, gx8, gxsf, ghsf, total;
+    int64_t ustart, row_of, gx8, gxsf, ghsf, slot_of, idx_slot, total;
     int64_t nblk, max_tiles;
 };
 static const int kPermuteBlock = 256;  // slots per permute block
@@ -87,7 +87,8 @@ static inline WsLayout ws_layout(const moe_dims &d) {
     w.nblk = (S + kPermuteBlock - 1) / kPermuteBlock;
     int64_t o = 0;
     auto take = [&](int64_t bytes) { const int64_t r = o; o = al256(o + bytes); return r; };
-    w.logits = take(T * E * 4);
+    w.logits = take(T * E * 4);  // router logits (the tensor-core router: its approximate logits)
+    w.rnorm = take(E * 4);       // router rows' 2-norms (tensor-core router)
     w.topk_idx = take(S * 4);
     w.topk_w = take(S * 4);
     w.counts = take(E * 4);
@@ -117,6 +118,9 @@ static inline WsLayout ws_layout(const moe_dims &d) {
     w.gx8 = take(S * dm);
     w.gxsf = take(w.max_tiles * (dm / 128) * 512);
     w.ghsf = take(w.max_tiles * (F / 128) * 512);
+    // expert cache: expert -> slot map of the current wave, slot of every top-k entry
+    w.slot_of = take(E * 4);
+    w.idx_slot = take(S * 4);
     w.total = o;
     return w;
 }

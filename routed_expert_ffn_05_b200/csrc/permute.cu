@@ -12,18 +12,24 @@ namespace moe {
 
 constexpr int kWarps = kPermuteBlock / 32;
 
-// Block b counts the experts of slots [b*256, b*256 + 256).
+// Block b counts the experts of slots [b*256, b*256 + 256). Expert ids are
+// taken relative to ebase: a slot whose id - ebase is outside [0, E) gets no
+// row; it is an error (reported through err) unless err is null, which is how
+// the expert-parallel layer drops the experts another rank owns.
 __global__ void __launch_bounds__(kPermuteBlock) permute_hist_kernel(const int32_t *__restrict__ idx,
-                                                                     int64_t S, int E,
+                                                                     int64_t S, int E, int ebase,
                                                                      int32_t *__restrict__ blkcnt, int *err) {
     extern __shared__ int32_t hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     const int64_t s = (int64_t)blockIdx.x * kPermuteBlock + threadIdx.x;
     if (s < S) {
-        const int e = idx[s];
-        if (e < 0 || e >= E) set_device_error(err, MOE_DEVERR_EXPERT_RANGE);
-        else atomicAdd(&hist[e], 1);
+        const int e = idx[s] - ebase;
+        if (e < 0 || e >= E) {
+            if (err) set_device_error(err, MOE_DEVERR_EXPERT_RANGE);
+        } else {
+            atomicAdd(&hist[e], 1);
+        }
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) blkcnt[(int64_t)blockIdx.x * E + e] = hist[e];
@@ -95,7 +101,7 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(const int32_t *__res
 }
 
 __global__ void __launch_bounds__(kPermuteBlock) permute_scatter_kernel(
-    const int32_t *__restrict__ idx, int64_t S, int E, const int32_t *__restrict__ blkbase,
+    const int32_t *__restrict__ idx, int64_t S, int E, int ebase, const int32_t *__restrict__ blkbase,
     int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm) {
     extern __shared__ int32_t wcnt[];  // [kWarps][E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -104,7 +110,7 @@ __global__ void __launch_bounds__(kPermuteBlock) permute_scatter_kernel(
     const int64_t s = (int64_t)blockIdx.x * kPermuteBlock + threadIdx.x;
     int e = -1;
     if (s < S) {
-        e = idx[s];
+        e = idx[s] - ebase;
         if (e < 0 || e >= E) e = -1;
     }
     const unsigned same = __match_any_sync(0xffffffffu, e);
@@ -117,19 +123,21 @@ __global__ void __launch_bounds__(kPermuteBlock) permute_scatter_kernel(
         const int32_t row = blkbase[(int64_t)blockIdx.x * E + e] + rank;
         perm[row] = (int32_t)s;
         inv_perm[s] = row;
+    } else if (s < S) {
+        inv_perm[s] = -1;  // a slot with no valid (or no local) expert has no row
     }
 }
 
 cudaError_t launch_permute(const moe_dims &d, const int32_t *idx, int32_t *counts, int32_t *offsets,
                            int32_t *perm, int32_t *inv_perm, int32_t *blkcnt, int32_t *blkbase,
-                           int64_t nblk, cudaStream_t s) {
+                           int64_t nblk, cudaStream_t s, int ebase, bool foreign_ok) {
     const int64_t S = (int64_t)d.T * d.k;
     if (nblk > 0)
-        permute_hist_kernel<<<(unsigned)nblk, kPermuteBlock, d.E * 4, s>>>(idx, S, d.E, blkcnt,
-                                                                           device_error_word());
+        permute_hist_kernel<<<(unsigned)nblk, kPermuteBlock, d.E * 4, s>>>(
+            idx, S, d.E, ebase, blkcnt, foreign_ok ? nullptr : device_error_word());
     permute_scan_kernel<<<1, 1024, 0, s>>>(blkcnt, nblk, d.E, blkbase, counts, offsets);
     if (nblk > 0)
-        permute_scatter_kernel<<<(unsigned)nblk, kPermuteBlock, kWarps * d.E * 4, s>>>(idx, S, d.E, blkbase,
+        permute_scatter_kernel<<<(unsigned)nblk, kPermuteBlock, kWarps * d.E * 4, s>>>(idx, S, d.E, ebase, blkbase,
                                                                                       perm, inv_perm);
     count_launches(nblk > 0 ? 3 : 1);
     return cudaGetLastError();

@@ -28,6 +28,8 @@
 //    warps, a 4-stage mbarrier ring; every wait is bounded.
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -349,15 +351,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
 }
 
 // CTA 0: token tiles per expert (ceil(count / 128)) and their exclusive
-// prefix. The other CTAs invert perm: row_of[slot] = the row holding the slot
-// (row_of enters filled with -1, so a slot no row names stays -1).
+// prefix. The other CTAs invert perm over the rows that hold a slot
+// (offsets[E] of them; fewer than S only when some slot had no valid expert):
+// row_of[slot] = the row holding the slot (row_of enters filled with -1, so a
+// slot no row names stays -1).
 __global__ void __launch_bounds__(1024) tc_plan_kernel(const int32_t *__restrict__ offsets, int E,
                                                        int32_t *__restrict__ ustart,
                                                        const int32_t *__restrict__ perm, int S,
                                                        int32_t *__restrict__ row_of, int *err) {
     if (blockIdx.x > 0) {
         const int i = (blockIdx.x - 1) * blockDim.x + threadIdx.x;
-        if (i < S) {
+        if (i < min(S, offsets[E])) {
             const int slot = perm[i];
             if ((unsigned)slot < (unsigned)S) row_of[slot] = i;
             else set_device_error(err, MOE_DEVERR_PERM);
@@ -409,8 +413,11 @@ __global__ void __launch_bounds__(256) tc_gather_quant_kernel(const uint16_t *__
     const int S = T * k;
     if (lane < k) {  // slot (t, lane): its row, the row's token-tile atom base and place in the tile
         int row = row_of[(int64_t)t * k + lane];
-        if ((unsigned)row >= (unsigned)S) {
-            set_device_error(err, MOE_DEVERR_PERM);
+        const int nrows = min(S, offsets[E]);
+        // a slot without a row is an error only when every slot should have one
+        // (fewer rows: slots of experts another rank or another cache wave runs)
+        if (row >= nrows || (row < 0 && nrows == S)) set_device_error(err, MOE_DEVERR_PERM);
+        if (row < 0 || row >= nrows) {
             row = -1;
         } else {
             const int e = expert_of_row(offsets, E, row), r = row - offsets[e];
@@ -469,16 +476,16 @@ int tc_num_sms() {
 }
 
 cudaError_t tc_set_attrs() {
-    static bool done[64] = {false};
+    static std::atomic<bool> done[64];  // per device; a repeated set-up from racing threads is harmless
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (done[dev]) return cudaSuccess;
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(tc_ffn_kernel<kModeGU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)))
         return e;
     if ((e = cudaFuncSetAttribute(tc_ffn_kernel<kModeDN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)))
         return e;
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_release);
     return cudaSuccess;
 }
 
@@ -525,15 +532,29 @@ cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_
     else dn.out = out_rows;
     dn.err = g.err;
 
-    int32_t *row_of = reinterpret_cast<int32_t *>(ws + L.row_of);
-    if ((e = cudaMemsetAsync(row_of, 0xFF, (size_t)S * 4, s)) != cudaSuccess) return e;
-    tc_plan_kernel<<<1 + (S + 1023) / 1024, 1024, 0, s>>>(offsets, d.E, ustart, perm, S, row_of, g.err);
-    tc_gather_quant_kernel<<<(d.T + 7) / 8, 256, 0, s>>>(x, offsets, row_of, ustart, d.T, d.E, d.k, d.d_model, gx8,
-                                                         gxsf, g.err);
+    if ((e = launch_tc_gather(d, x, offsets, perm, ustart, reinterpret_cast<int32_t *>(ws + L.row_of), gx8, gxsf, s)))
+        return e;
     const int grid = tc_num_sms();
     tc_ffn_kernel<kModeGU><<<grid, kTcThreads, kTcSmemBytes, s>>>(g);
     tc_ffn_kernel<kModeDN><<<grid, kTcThreads, kTcSmemBytes, s>>>(dn);
-    count_launches(4);
+    count_launches(2);
+    return cudaGetLastError();
+}
+
+// The tensor-core path's activation staging: token-tile plan, slot -> row
+// inverse of perm, and the MXFP8 rows in expert order with their scale atoms
+// (gx8 [S][d], gxsf [tiles][d/128][512], ustart [E+1]).
+cudaError_t launch_tc_gather(const moe_dims &d, const uint16_t *x, const int32_t *offsets, const int32_t *perm,
+                             int32_t *ustart, int32_t *row_of, uint8_t *gx8, uint8_t *gxsf, cudaStream_t s) {
+    const int S = d.T * d.k;
+    if (S == 0) return cudaSuccess;
+    cudaError_t e;
+    int *err = device_error_word();
+    if ((e = cudaMemsetAsync(row_of, 0xFF, (size_t)S * 4, s)) != cudaSuccess) return e;
+    tc_plan_kernel<<<1 + (S + 1023) / 1024, 1024, 0, s>>>(offsets, d.E, ustart, perm, S, row_of, err);
+    tc_gather_quant_kernel<<<(d.T + 7) / 8, 256, 0, s>>>(x, offsets, row_of, ustart, d.T, d.E, d.k, d.d_model, gx8,
+                                                         gxsf, err);
+    count_launches(2);
     return cudaGetLastError();
 }
 

@@ -59,6 +59,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
+// The same, also giving up as soon as *abort (a CTA-wide flag another role of
+// the CTA sets when it fails) is non-zero. Not for waits on copies in flight,
+// which must always land before the CTA exits.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
 // Global -> shared bulk copy (16-byte aligned, size a multiple of 16) that
 // completes `bytes` of transaction count on `bar`.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

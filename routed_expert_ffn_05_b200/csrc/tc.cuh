@@ -1,5 +1,6 @@
 // 5th-generation tensor core (tcgen05) helpers for sm_100a: tensor-memory
-// allocation, block-scaled MMA (kind::mxf8f6f4), scale-factor copies into
+// allocation, block-scaled MMA (kind::mxf8f6f4), bf16 MMA (kind::f16),
+// scale-factor copies into
 // tensor memory, tensor-memory loads, and the shared-memory matrix
 // descriptors these instructions read.
 #pragma once
@@ -53,6 +54,17 @@ __device__ __forceinline__ void tc_mma_mx(uint32_t d, uint64_t adesc, uint64_t b
         : "memory");
 }
 
+// D[M][N] (+)= A[M][K] . B[N][K]^T with K = 16 bf16 elements, fp32 accumulate
+// in TMEM; A and B in shared memory (descriptors).
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Thread i of the warp reads TMEM lane (lane field of taddr) + i, columns
 // taddr .. taddr + 31 (one 32-bit value per column).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -93,6 +105,12 @@ __device__ __forceinline__ uint64_t sdesc_sf(const void *p) {
 __host__ __device__ constexpr uint32_t idesc_mx(int a_fmt, int b_fmt, int M, int N) {
     return (uint32_t)(a_fmt & 7) << 7 | (uint32_t)(b_fmt & 7) << 10 | (uint32_t)(N >> 3) << 17 | 1u << 23 |
            (uint32_t)(M >> 4) << 24;
+}
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
+// fp32 accumulator: D format 1 (bits 4..5), A and B format 1 = bf16 (bits
+// 7..9, 10..12), N / 8 (bits 17..22), M / 16 (bits 24..28).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return 1u << 4 | 1u << 7 | 1u << 10 | (uint32_t)(N >> 3) << 17 | (uint32_t)(M >> 4) << 24;
 }
 __device__ __forceinline__ uint32_t idesc_sf_ids(uint32_t idesc, uint32_t a_id, uint32_t b_id) {
     return idesc | (b_id & 3u) << 4 | (a_id & 3u) << 29;

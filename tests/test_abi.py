@@ -100,3 +100,17 @@ def test_binding_structs_match_the_header():
     import routed_expert_ffn_05_b200 as M
     assert [f for f, _ in M.moe_dims._fields_] == header_struct_fields("moe_dims")
     assert [f for f, _ in M.moe_weights._fields_] == header_struct_fields("moe_weights")
+    assert [f for f, _ in M.moe_cache_stats._fields_] == header_struct_fields("moe_cache_stats")
+
+
+def test_static_ws_bound_matches_its_documentation():
+    """The header says moe_layer_static_ws holds T = 97 decode tokens (d_model
+    4096, d_ff 2048, E 256, k 8, shared d_ff 2048): the workspace of T = 97
+    fits the built-in array and that of T = 98 does not."""
+    import routed_expert_ffn_05_b200 as M
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    mib = int(re.search(r"#define MOE_STATIC_WS_BYTES \((\d+)u << 20\)", src).group(1))
+    assert M.MOE_STATIC_WS_BYTES == mib << 20
+    documented = int(re.search(r"holds up to T = (\d+) tokens", src).group(1))
+    ws = lambda T: M.moe_workspace_size(M.make_dims(T, 4096, 2048, 256, 8, d_ff_shared=2048))
+    assert ws(documented) <= M.MOE_STATIC_WS_BYTES < ws(documented + 1)

@@ -49,7 +49,7 @@ def cfg_of(name, T=None):
 
 
 LAYER_CASES = [("tiny", None), ("decode", 1), ("decode", 2), ("decode", 4), ("decode", 8),
-               ("q2k", 1), ("q2k", 8), ("prefill", None), ("hash", None)]
+               ("q2k", 1), ("q2k", 8), ("q2k", 16), ("prefill", None), ("hash", None)]
 _cases = {}
 
 
@@ -61,12 +61,29 @@ def get_case(name, T=None):
     return _cases[key]
 
 
-def sample_tokens(cfg, n=48, seed=0):
+def tile_edge_rows(offsets, tile=128):
+    """Per expert with rows: the first and last row of its last 128-row token
+    tile (the partial tile, when the count is not a multiple of 128)."""
+    out = []
+    for e in range(len(offsets) - 1):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            out += [lo + (hi - lo - 1) // tile * tile, hi - 1]
+    return np.unique(np.array(out, np.int64))
+
+
+def sample_tokens(cfg, ora_idx=None, n=512, seed=0):
+    """All tokens of a small batch; else n random tokens, the first and last,
+    and the tokens of the first and last row of every expert's last token tile."""
     if cfg.T <= n:
         return np.arange(cfg.T, dtype=np.int32)
     rng = np.random.default_rng(seed)
     s = rng.choice(cfg.T, n - 2, replace=False)
-    return np.unique(np.concatenate([[0, cfg.T - 1], s])).astype(np.int32)
+    extra = []
+    if ora_idx is not None:
+        _, offsets, perm, _ = oracle.permute(ora_idx, cfg.E)
+        extra = perm[tile_edge_rows(offsets)] // cfg.k
+    return np.unique(np.concatenate([[0, cfg.T - 1], s, extra])).astype(np.int32)
 
 
 # ---- formats ----------------------------------------------------------------
@@ -172,8 +189,10 @@ def test_route_bitexact(name, T):
     np.testing.assert_allclose(host(w), c.ora_w, rtol=0, atol=2e-6)
 
 
-def test_route_ties_to_lower_index():
-    cfg = synth.LayerConfig("ties", T=8, d=256, F=256, E=16, k=4)
+@pytest.mark.parametrize("T", [8, 40])
+def test_route_ties_to_lower_index(T):
+    """T = 8 runs the per-token router, T = 40 the batch router on the tensor cores."""
+    cfg = synth.LayerConfig("ties", T=T, d=256, F=256, E=16, k=4)
     wr = synth.make_router(cfg)
     wr[5] = wr[2]            # experts 2 and 5 always tie
     wr[9] = wr[2]
@@ -254,11 +273,12 @@ def test_expert_ffn(name, T):
     S = cfg.T * cfg.k
     if S <= 64:
         ranges = [(0, S)]
-    else:  # rows from the busiest expert, the last expert, and random places
+    else:  # rows from the busiest expert, the last expert, random places, every expert's last tile edges
         e_big = int(np.argmax(np.diff(offsets_r)))
         rng = np.random.default_rng(3)
-        starts = [offsets_r[e_big], S - 4] + list(rng.integers(0, S - 4, 10))
+        starts = [offsets_r[e_big], S - 4] + list(rng.integers(0, S - 4, 64))
         ranges = [(int(s), int(s) + 4) for s in starts]
+        ranges += [(int(r), int(r) + 1) for r in tile_edge_rows(offsets_r)]
     for a, b in ranges:
         ref = oracle.expert_ffn_rows(c.ora, c.x, offsets_r, perm_r, a, b)
         assert_rel(got[a:b], ref, TOL[cfg.act], f"{name} rows {a}:{b}")
@@ -293,7 +313,7 @@ def test_layer(name, T):
     y = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device=DEV)
     M.moe_layer(c.dims, c.weights, c.x_d, c.tok_d, y, c.ws)
     assert M.moe_get_device_error() == 0
-    toks = sample_tokens(cfg)
+    toks = sample_tokens(cfg, c.ora_idx)
     idx, w, ref = oracle.layer_tokens(c.ora, c.x, toks, c.token_ids)
     np.testing.assert_array_equal(idx, c.ora_idx[toks])
     assert_rel(host(y)[toks], ref, TOL[cfg.act], f"{name} T={cfg.T}")
