@@ -6,9 +6,9 @@ uses it and shares no code with it. Each C function cites the definition it
 follows (see ``oracle.h`` and the ``*.c`` files).
 
 Parity status: every function is pinned by a ``-m "not gpu"`` test against the
-format definitions, brute force, closed forms or an independently coded dense
-FFN, except the SplitMix64 finaliser constants inside hash routing, which are
-pinned only by properties (bijectivity, uniformity, distinctness).
+format definitions, brute force, closed forms, library routines or an
+independently coded dense FFN; the SplitMix64 draws of hash routing are pinned
+draw by draw against a library implementation of the generator.
 """
 from __future__ import annotations
 
@@ -23,7 +23,7 @@ _SRCS = ["formats.c", "route.c", "permute.c", "ffn.c"]
 _SO = os.path.join(_HERE, "liboracle.so")
 
 W_MXFP4, W_Q2K = 1, 2
-A_BF16, A_MXFP8 = 0, 1
+A_BF16, A_MXFP8, A_MXFP4 = 0, 1, 2
 ROUTE_SOFTMAX, ROUTE_HASH = 0, 1
 Q2K_BLOCK, Q2K_BYTES = 256, 84
 MAX_DRAWS = 1024
@@ -67,6 +67,7 @@ def lib():
             "ora_f64_to_bf16": (u16, [f64]), "ora_bf16_value": (f64, [u16]),
             "ora_mxfp4_quantize": (None, [vp, i64, i64, vp, vp]),
             "ora_mxfp4_dequantize": (None, [vp, vp, i64, i64, vp]),
+            "ora_mxfp4_quantize_f64": (None, [vp, i64, i64, vp, vp]),
             "ora_mxfp8_quantize_f64": (None, [vp, i64, i64, vp, vp]),
             "ora_mxfp8_quantize_bf16": (None, [vp, i64, i64, vp, vp]),
             "ora_mxfp8_dequantize": (None, [vp, vp, i64, i64, vp]),
@@ -164,6 +165,16 @@ def mxfp4_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     lib().ora_mxfp4_dequantize(_p(np.ascontiguousarray(codes)), _p(np.ascontiguousarray(scales)),
                                rows, K, _p(out))
     return out
+
+
+def mxfp4_quantize_f64(v: np.ndarray):
+    """fp64 [rows][K] -> (codes u8 [rows][K/2], scales u8 [rows][K/32]), the weights' MXFP4 rule."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    rows, K = v.shape
+    codes = np.empty((rows, K // 2), np.uint8)
+    scales = np.empty((rows, K // 32), np.uint8)
+    lib().ora_mxfp4_quantize_f64(_p(v), rows, K, _p(codes), _p(scales))
+    return codes, scales
 
 
 def mxfp8_quantize_f64(v: np.ndarray):
@@ -278,7 +289,7 @@ class LayerWeights:
         s = Layer()
         s.T, s.d, s.F, s.E, s.k = c.T, c.d, c.F, c.E, c.k
         s.wfmt = W_Q2K if c.wfmt == "q2k" else W_MXFP4
-        s.act = A_MXFP8 if c.act == "mxfp8" else A_BF16
+        s.act = {"mxfp8": A_MXFP8, "mxfp4": A_MXFP4}.get(c.act, A_BF16)
         s.route = ROUTE_HASH if c.route == "hash" else ROUTE_SOFTMAX
         s.Fs = c.Fs if self.sw1 is not None else 0
         s.max_draws = MAX_DRAWS

@@ -15,7 +15,10 @@
  * Readings (the pages are silent):
  *  - bf16-activation mode ("w4a16"): a = x (bf16) and h is rounded to bf16
  *    before W2; MXFP8 mode ("w4a8"): a is x quantised to MXFP8 along d and h
- *    is quantised to MXFP8 along F before W2;
+ *    is quantised to MXFP8 along F before W2; MXFP4 mode ("w4a4", both
+ *    operands on the FP4 matrix instructions the pages name for Blackwell,
+ *    "DwarfStar", hysenlabs.com, "Model support and quantisation"): the same
+ *    with MXFP4 (E2M1 elements, the weights' rule);
  *  - the shared expert always takes bf16 x and rounds h to bf16; its gate is 1.
  * Arithmetic is fp64; MXFP4 dots sum each 32-element block, then apply the
  * block scale.
@@ -83,6 +86,18 @@ static void mxfp8_roundtrip(double *v, int K) {
     free(s);
 }
 
+/* The same with MXFP4 (w4a4 activations). */
+static void mxfp4_roundtrip(double *v, int K) {
+    uint8_t *c = (uint8_t *)malloc((size_t)K / 2), *s = (uint8_t *)malloc((size_t)K / 32);
+    float *f = (float *)malloc(sizeof(float) * (size_t)K);
+    ora_mxfp4_quantize_f64(v, 1, K, c, s);
+    ora_mxfp4_dequantize(c, s, 1, K, f);  /* E2M1 x 2^e: exact in fp32 */
+    for (int i = 0; i < K; ++i) v[i] = (double)f[i];
+    free(c);
+    free(s);
+    free(f);
+}
+
 void ora_expert_ffn_token(const ora_layer *L, int e, const uint16_t *x_t, double *o) {
     const int d = L->d, F = L->F;
     double lut[16];
@@ -91,6 +106,7 @@ void ora_expert_ffn_token(const ora_layer *L, int e, const uint16_t *x_t, double
     double *h = (double *)malloc(sizeof(double) * (size_t)F);
     for (int i = 0; i < d; ++i) a[i] = ora_bf16_value(x_t[i]);
     if (L->act == ORA_A_MXFP8) mxfp8_roundtrip(a, d);
+    if (L->act == ORA_A_MXFP4) mxfp4_roundtrip(a, d);
 
     const int64_t eF = (int64_t)e * F, ed = (int64_t)e * d;
     for (int n = 0; n < F; ++n) {
@@ -99,6 +115,7 @@ void ora_expert_ffn_token(const ora_layer *L, int e, const uint16_t *x_t, double
         h[n] = silu(g) * u;
     }
     if (L->act == ORA_A_MXFP8) mxfp8_roundtrip(h, F);
+    else if (L->act == ORA_A_MXFP4) mxfp4_roundtrip(h, F);
     else
         for (int n = 0; n < F; ++n) h[n] = ora_bf16_value(ora_f64_to_bf16(h[n]));
     for (int i = 0; i < d; ++i) o[i] = dot_expert(L, L->w2, L->w2s, ed + i, h, F, lut);

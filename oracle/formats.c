@@ -176,29 +176,41 @@ static int mx_shared_exp(double amax, int emax_elem) {
     return se;
 }
 
+/* One MXFP4 block of 32 values: 16 code bytes (element 2i in the low
+ * nibble) and the E8M0 scale byte. */
+static uint8_t mxfp4_block(const double *v, uint8_t *c) {
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(v[i]));
+    if (amax == 0.0) {
+        memset(c, 0, 16);
+        return 127;
+    }
+    const int se = mx_shared_exp(amax, 2);
+    for (int i = 0; i < 32; i += 2) {
+        const uint8_t lo = ora_e2m1_encode(ldexp(v[i], -se));
+        const uint8_t hi = ora_e2m1_encode(ldexp(v[i + 1], -se));
+        c[i / 2] = (uint8_t)(lo | (hi << 4));
+    }
+    return (uint8_t)(se + 127);
+}
+
 void ora_mxfp4_quantize(const float *w, int64_t rows, int64_t K, uint8_t *codes, uint8_t *scales) {
     const int64_t nb = K / 32;
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
+        double buf[32];
         for (int64_t b = 0; b < nb; ++b) {
-            const float *v = w + r * K + b * 32;
-            uint8_t *c = codes + r * (K / 2) + b * 16;
-            double amax = 0.0;
-            for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs((double)v[i]));
-            if (amax == 0.0) {
-                scales[r * nb + b] = 127;
-                memset(c, 0, 16);
-                continue;
-            }
-            const int se = mx_shared_exp(amax, 2);
-            scales[r * nb + b] = (uint8_t)(se + 127);
-            for (int i = 0; i < 32; i += 2) {
-                const uint8_t lo = ora_e2m1_encode(ldexp((double)v[i], -se));
-                const uint8_t hi = ora_e2m1_encode(ldexp((double)v[i + 1], -se));
-                c[i / 2] = (uint8_t)(lo | (hi << 4));
-            }
+            for (int i = 0; i < 32; ++i) buf[i] = (double)w[r * K + b * 32 + i];
+            scales[r * nb + b] = mxfp4_block(buf, codes + r * (K / 2) + b * 16);
         }
     }
+}
+
+void ora_mxfp4_quantize_f64(const double *v, int64_t rows, int64_t K, uint8_t *codes, uint8_t *scales) {
+    const int64_t nb = K / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < nb; ++b)
+            scales[r * nb + b] = mxfp4_block(v + r * K + b * 32, codes + r * (K / 2) + b * 16);
 }
 
 void ora_mxfp4_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K,

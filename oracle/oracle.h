@@ -49,6 +49,8 @@ double ora_bf16_value(uint16_t b);
 void ora_mxfp4_quantize(const float *w, int64_t rows, int64_t K, uint8_t *codes, uint8_t *scales);
 void ora_mxfp4_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t rows, int64_t K,
                           float *out);
+/* The same rule on fp64 values (MXFP4 activations, "w4a4"). */
+void ora_mxfp4_quantize_f64(const double *v, int64_t rows, int64_t K, uint8_t *codes, uint8_t *scales);
 /* MXFP8 (E4M3 elements): codes [rows][K], scales [rows][K/32]. */
 void ora_mxfp8_quantize_f64(const double *v, int64_t rows, int64_t K, uint8_t *codes,
                             uint8_t *scales);
@@ -76,7 +78,7 @@ int ora_permute(const int32_t *idx, int T, int k, int E, int32_t *counts, int32_
 
 /* ---- expert FFN, combine, layer (ffn.c) -------------------------------- */
 enum { ORA_W_MXFP4 = 1, ORA_W_Q2K = 2 };
-enum { ORA_A_BF16 = 0, ORA_A_MXFP8 = 1 };
+enum { ORA_A_BF16 = 0, ORA_A_MXFP8 = 1, ORA_A_MXFP4 = 2 };
 enum { ORA_ROUTE_SOFTMAX = 0, ORA_ROUTE_HASH = 1 };
 
 typedef struct {

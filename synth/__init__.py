@@ -162,7 +162,7 @@ class LayerConfig:
     E: int = 256
     k: int = 8
     route: str = "softmax"      # "softmax" (top-k softmax) | "hash"
-    act: str = "bf16"           # "bf16" (w4a16) | "mxfp8" (w4a8)
+    act: str = "bf16"           # "bf16" (w4a16) | "mxfp8" (w4a8) | "mxfp4" (w4a4)
     wfmt: str = "mxfp4"         # "mxfp4" | "q2k"
     Fs: int = 0                 # shared-expert d_ff; 0 = no shared expert
     zipf_s: float = 0.0         # >0: router bias gives Zipf(zipf_s) expert popularity

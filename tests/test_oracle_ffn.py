@@ -36,16 +36,39 @@ def mxfp8_roundtrip(v):
     return (q * X).reshape(v.shape)
 
 
+E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])  # OCP MX v1.0 E2M1 magnitudes, codes 0..7
+
+
+def mxfp4_roundtrip(v):
+    """MX FP4 (E2M1) quantise-dequantise along the last axis, 32-blocks, by
+    brute force over the format's eight magnitudes: the nearest one, a tie to
+    the even code (mantissa bit 0), values past 6 to 6; scale 2^(floor(log2
+    amax) - 2) as for the weights."""
+    v = np.asarray(v, np.float64)
+    blk = v.reshape(*v.shape[:-1], -1, 32)
+    amax = np.abs(blk).max(axis=-1, keepdims=True)
+    e = np.frexp(np.where(amax > 0, amax, 1.0))[1] - 1 - 2
+    X = np.exp2(np.clip(e, -127, 127))
+    y = blk / X
+    dist = np.abs(np.abs(y)[..., None] - E2M1_MAG)
+    best = dist == dist.min(axis=-1, keepdims=True)
+    even = best & (np.arange(8) % 2 == 0)
+    pick = np.where(even.any(axis=-1), np.argmax(even, axis=-1), np.argmax(best, axis=-1))
+    q = np.where(amax > 0, np.sign(y) * E2M1_MAG[pick], 0.0)
+    return (q * X).reshape(v.shape)
+
+
 def silu(g):
     return g / (1 + np.exp(-g))
 
 
 def dense_ffn(a, W1, W3, W2, act="bf16"):
-    if act == "mxfp8":
-        a = mxfp8_roundtrip(a)
+    roundtrip = {"mxfp8": mxfp8_roundtrip, "mxfp4": mxfp4_roundtrip}.get(act)
+    if roundtrip:
+        a = roundtrip(a)
     g, u = W1 @ a, W3 @ a
     h = silu(g) * u
-    h = mxfp8_roundtrip(h) if act == "mxfp8" else to_bf16(h)
+    h = roundtrip(h) if roundtrip else to_bf16(h)
     return W2 @ h
 
 
@@ -79,7 +102,7 @@ def rand_x(rng, T, d):
         torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("act", ["bf16", "mxfp8"])
+@pytest.mark.parametrize("act", ["bf16", "mxfp8", "mxfp4"])
 def test_dense_equivalence_single_expert(ora, syn, act):
     """E = 1, k = 1: the MoE layer is exactly one dense SwiGLU FFN."""
     cfg = syn.LayerConfig("t", T=3, d=256, F=512, E=1, k=1, act=act)
@@ -90,7 +113,7 @@ def test_dense_equivalence_single_expert(ora, syn, act):
     assert np.all(idx == 0) and np.all(w == 1.0)
     for t in range(3):
         ref = dense_ffn(bf16_vals(x[t]), W1[0], W3[0], W2[0], act)
-        tol = (1e-4 if act == "bf16" else 3e-3) * np.abs(ref).max()
+        tol = {"bf16": 1e-4, "mxfp8": 3e-3, "mxfp4": 1e-6}[act] * np.abs(ref).max()
         np.testing.assert_allclose(y[t], ref, rtol=0, atol=tol)
         o = ora.expert_ffn_token(L, 0, x[t])
         np.testing.assert_allclose(o, ref, rtol=0, atol=tol)
@@ -186,3 +209,23 @@ def test_combine_closed_forms(ora):
     sh = rng.normal(0, 1, (T, d)).astype(np.float32)
     ref = np.einsum("tk,tkd->td", w.astype(np.float64), rows[inv.reshape(T, k)].astype(np.float64)) + sh
     np.testing.assert_allclose(ora.combine(rows, inv, w, sh), ref, rtol=1e-6, atol=1e-6)
+
+
+def test_mxfp4_activation_quantiser_vs_brute_force(ora):
+    """The fp64 MXFP4 quantiser (w4a4 activations) decodes to the brute-force
+    nearest-value roundtrip above, over six decades, zero blocks and exact
+    ties; on fp32 inputs it writes the bytes of the weights' quantiser."""
+    rng = np.random.default_rng(23)
+    v = rng.normal(0, 1, (64, 256)) * np.exp2(rng.integers(-20, 20, (64, 1)))
+    v[0, :32] = 0.0
+    v[1, :32] = np.tile([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 4.0], 4) * rng.choice([-1, 1], 32)  # ties at scale 1
+    v[1, 0] = 6.0 * 1.0  # amax 6: scale 2^0
+    v[2, :32] = 7.0 * rng.choice([-1, 1], 32)
+    codes, scales = ora.mxfp4_quantize_f64(v)
+    dec = ora.mxfp4_dequantize(codes, scales).astype(np.float64)
+    np.testing.assert_array_equal(dec, mxfp4_roundtrip(v))
+    f = v.astype(np.float32)
+    c32, s32 = ora.mxfp4_quantize(f)
+    c64, s64 = ora.mxfp4_quantize_f64(f.astype(np.float64))
+    np.testing.assert_array_equal(c32, c64)
+    np.testing.assert_array_equal(s32, s64)
