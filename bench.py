@@ -113,7 +113,7 @@ class DeviceLayer:
         M, cfg = self.M, self.cfg
         return M.make_dims(T, cfg.d, cfg.F, cfg.E, cfg.k,
                            M.MOE_ROUTE_HASH if cfg.route == "hash" else M.MOE_ROUTE_SOFTMAX_TOPK,
-                           M.MOE_A_MXFP8 if cfg.act == "mxfp8" else M.MOE_A_BF16,
+                           {"mxfp8": M.MOE_A_MXFP8, "mxfp4": M.MOE_A_MXFP4}.get(cfg.act, M.MOE_A_BF16),
                            M.MOE_W_Q2K if cfg.wfmt == "q2k" else M.MOE_W_MXFP4,
                            cfg.Fs if cfg.Fs else 0)
 
@@ -396,7 +396,7 @@ def workload_desc(cfg):
     route = "hash (SplitMix64 of the token id)" if cfg.route == "hash" else f"top-{cfg.k} softmax"
     if cfg.zipf_s:
         route += f", Zipf({cfg.zipf_s}) router bias"
-    act = "MXFP8 activations (w4a8)" if cfg.act == "mxfp8" else "bf16 activations"
+    act = {"mxfp8": "MXFP8 activations (w4a8)", "mxfp4": "MXFP4 activations (w4a4)"}.get(cfg.act, "bf16 activations")
     sh = f", bf16 shared expert d_ff {cfg.Fs}" if cfg.Fs else ""
     return (f"{cfg.name} layer T={cfg.T}: d_model {cfg.d}, d_ff {cfg.F}, {cfg.E} {fmt} routed experts, "
             f"{route} routing, {act}{sh}")
@@ -420,6 +420,8 @@ def main():
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--act", default=None, choices=["bf16", "mxfp8", "mxfp4"],
+                    help="activation mode override (w4a16 / w4a8 / w4a4)")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism: the N ranks split one layer's routed experts (one batch, "
                          "partial sums all-reduced) instead of running N replicas")
@@ -433,6 +435,8 @@ def main():
     E = args.E if args.E else base_cfg.E
     T = args.T if args.T else base_cfg.T
     cfg = replace(base_cfg.with_T(T), E=E)
+    if args.act:
+        cfg = replace(cfg, act=args.act)
     workload = workload_desc(cfg)
     n_cpu_tokens = min(T, 8)
 
@@ -494,13 +498,17 @@ def main():
     # roofline of the expert FFN (the dominant stage), per step
     hbm, bf16, src = peaks()
     ffn_ms = statistics.mean(r["ffn_ms"]) if r["ffn_ms"] else float("nan")
-    if cfg.act == "mxfp8":  # a dense contraction on the FP8 tensor-core rate
+    if cfg.act in ("mxfp8", "mxfp4") or T > 8:  # a dense contraction at the FP8 / FP4 / bf16 tensor-core rate
         fl = expert_flops(cfg, T)
         achieved = fl / (ffn_ms / 1000.0) / 1e12
-        peak = 2.0 * bf16  # E4M3 x E2M1 runs at the FP8 rate: 2x bf16 dense (nominal ratio)
+        ratio = {"mxfp8": 2.0, "mxfp4": 4.0}.get(cfg.act, 1.0)  # nominal dense ratios to bf16: FP8 2x, FP4 4x
+        peak = ratio * bf16
         roof = {"kernel": "expert FFN: plan + gather/quantise + gate/up GEMM + down GEMM (tcgen05)",
                 "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_source": f"{src} bf16 x 2 (FP8 nominal ratio)",
+                "frac": achieved / peak,
+                "peak_source": f"{src} bf16" + (f" x {ratio:g} ({'FP8' if ratio == 2 else 'FP4'} nominal ratio)"
+                                                 if ratio != 1 else ""),
+                "frac_of_fp4_peak": achieved / (4.0 * bf16),
                 "traffic": None, "algorithmic_flops": fl, "ffn_ms": ffn_ms}
     else:
         xb = torch.from_numpy(synth.make_x(cfg, 0, 1000 * (0 if ep else rank)).astype(np.int16)).cuda()
@@ -520,8 +528,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "strong" if ep else "weak",
         "vs_baseline": None,
-        "dtype": ("mxfp4 x mxfp8 -> fp32" if cfg.act == "mxfp8" else
-                  ("q2k x bf16 -> fp32" if cfg.wfmt == "q2k" else "mxfp4 x bf16 -> fp32")),
+        "dtype": ("mxfp4 x mxfp8 -> fp32" if cfg.act == "mxfp8" else "mxfp4 x mxfp4 -> fp32" if cfg.act == "mxfp4"
+                  else ("q2k x bf16 -> fp32" if cfg.wfmt == "q2k" else "mxfp4 x bf16 -> fp32")),
         "data": "synthetic",
         "config": {"workload": workload, "T": T, "batches": NBATCH,
                    "l2": "flushed between steps (256 MB write), flush outside the timed events",
@@ -546,13 +554,17 @@ def main():
                 bd[f"decode_T{Tb}"] = {"tokens_per_s": Tb / (statistics.mean(rr["ms"]) / 1000),
                                        "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"]),
                                        **hbm_fraction(M, torch, lb, dec.with_T(Tb), Tb, rr, hbm, rank)}
-            for name in ("prefill", "hash"):
-                c = replace(synth.CONFIGS[name], E=E)
+            for name, act in (("prefill", "mxfp8"), ("hash", "mxfp8"), ("prefill", "mxfp4"), ("hash", "mxfp4"),
+                              ("prefill", "bf16")):
+                c = replace(synth.CONFIGS[name], E=E, act=act)
                 rr = measure(M, torch, base.with_weights(c), c.T, 3, 3, rank, 1, batches=2)
                 fl = expert_flops(c, c.T)
-                bd[name] = {"T": c.T, "tokens_per_s": c.T / (statistics.mean(rr["ms"]) / 1000),
-                            "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"]),
-                            "ffn_tflops": fl / (statistics.mean(rr["ffn_ms"]) / 1000) / 1e12}
+                tf = fl / (statistics.mean(rr["ffn_ms"]) / 1000) / 1e12
+                bd[name + {"mxfp8": "", "mxfp4": "_w4a4", "bf16": "_w4a16"}[act]] = {
+                    "T": c.T, "act": act, "tokens_per_s": c.T / (statistics.mean(rr["ms"]) / 1000),
+                    "ms": statistics.mean(rr["ms"]), "ffn_ms": statistics.mean(rr["ffn_ms"]), "ffn_tflops": tf,
+                    "ffn_frac_of_own_peak": tf / ({"mxfp8": 2.0, "mxfp4": 4.0, "bf16": 1.0}[act] * bf16),
+                    "ffn_frac_of_fp4_peak": tf / (4.0 * bf16)}
             del base
             torch.cuda.empty_cache()
             q2 = DeviceLayer(M, torch, replace(synth.CONFIGS["q2k"], E=E))

@@ -64,9 +64,15 @@ typedef enum {
 
 /* Routed-expert weight format. */
 typedef enum { MOE_W_MXFP4 = 1, MOE_W_Q2K = 2 } moe_wfmt;
-/* Activation mode of the routed experts: bf16 ("w4a16") or MXFP8 E4M3 with
- * per-32 E8M0 scales ("w4a8"; x and the hidden h are both quantised). */
-typedef enum { MOE_A_BF16 = 0, MOE_A_MXFP8 = 1 } moe_amode;
+/* Activation mode of the routed experts: bf16 ("w4a16"), MXFP8 E4M3 with
+ * per-32 E8M0 scales ("w4a8"), or MXFP4 E2M1 with per-32 E8M0 scales ("w4a4",
+ * both GEMM operands on the FP4 matrix instructions that "DwarfStar",
+ * hysenlabs.com, "Model support and quantisation", names for Blackwell). In
+ * the quantised modes x and the hidden h are both quantised along their
+ * length, by the rule the weights use (scale 2^(floor(log2 amax) - emax),
+ * emax 8 for E4M3 and 2 for E2M1; elements round to nearest even and
+ * saturate). */
+typedef enum { MOE_A_BF16 = 0, MOE_A_MXFP8 = 1, MOE_A_MXFP4 = 2 } moe_amode;
 /* Routing: top-k of bf16 router logits with softmax gates, or hash routing. */
 typedef enum { MOE_ROUTE_SOFTMAX_TOPK = 0, MOE_ROUTE_HASH = 1 } moe_rmode;
 

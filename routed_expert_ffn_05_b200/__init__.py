@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE, MOE_ERR_TIMEOUT = range(6)
 # formats and modes
 MOE_W_MXFP4, MOE_W_Q2K = 1, 2
-MOE_A_BF16, MOE_A_MXFP8 = 0, 1
+MOE_A_BF16, MOE_A_MXFP8, MOE_A_MXFP4 = 0, 1, 2
 MOE_ROUTE_SOFTMAX_TOPK, MOE_ROUTE_HASH = 0, 1
 MOE_MAT_W1, MOE_MAT_W2, MOE_MAT_W3 = 1, 2, 3
 MOE_DEVERR_NONE, MOE_DEVERR_EXPERT_RANGE, MOE_DEVERR_HASH_CAP, MOE_DEVERR_TIMEOUT, MOE_DEVERR_PERM = range(5)

@@ -52,7 +52,7 @@ static moe_status check_dims(const moe_dims *d) {
     if (d->E > 1024 || d->k > 32 || d->k > d->E) return MOE_ERR_INVALID_ARG;
     if ((int64_t)d->T * d->k >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
     if (d->route != MOE_ROUTE_SOFTMAX_TOPK && d->route != MOE_ROUTE_HASH) return MOE_ERR_INVALID_ARG;
-    if (d->act != MOE_A_BF16 && d->act != MOE_A_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (d->act != MOE_A_BF16 && d->act != MOE_A_MXFP8 && d->act != MOE_A_MXFP4) return MOE_ERR_INVALID_ARG;
     if (d->wfmt != MOE_W_MXFP4 && d->wfmt != MOE_W_Q2K) return MOE_ERR_INVALID_ARG;
     if (d->d_ff_shared < 0 || d->d_ff_shared % 256) return MOE_ERR_INVALID_ARG;
     return MOE_OK;

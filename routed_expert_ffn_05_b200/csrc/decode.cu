@@ -170,11 +170,12 @@ __device__ __forceinline__ int active_experts(const int32_t *offsets, int E, int
 }
 
 // Unit numbering: [shared gate/up][routed gate/up][shared down][routed down].
-// Shared gate/up units are assigned statically (they need no routing), routed
-// gate/up units through the work queue, and the down units as one contiguous,
-// stage-balanced range per CTA (few expert changes, so few reloads of h).
-// A routed gate/up unit is 16 rows of W1 and W3 over all K: two stages of
-// MXFP4 codes, or one stage of Q2_K quants (half the bytes).
+// The shared gate/up units need no routing: they stream while the routing
+// kernels run. The shared down units sit between the two routed phases, where
+// they need no wait (every shared gate/up tile is long done) and cover the
+// tail of the routed gate/up phase. A routed gate/up unit is 16 rows of W1 and
+// W3 over all K: two stages of MXFP4 codes, or one stage of Q2_K quants (half
+// the bytes).
 template <int WF> constexpr int gu_stages() { return WF == MOE_W_Q2K ? 1 : 2; }
 
 template <int WF>
@@ -509,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             prefetch_tensormap(&a.m2c);
             t = (int)atomicAdd(ticket, 1u);
             while (t < usg && !s.abort) {
-                const int nt = (int)atomicAdd(ticket, 1u);  // the next claim is fetched one chunk ahead
+                const int nt = (int)atomicAdd(ticket, 1u);  // the next claim is fetched one unit ahead
                 issue(t, unit_of<WF>(t, usg, 0, 0));
                 t = nt;
             }
@@ -535,9 +536,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         const int cb = (R - R / 4) / G;
         const int nb = cb >= kGrab ? G : 0;
         const int t_small = usg + nb, t_dn = t_small + (R - nb * cb + kGrab - 1) / kGrab;
-        // Down tickets: G contiguous ranges of equal cost (shared tiles cost 2
-        // stages, routed ones dn_stages), so a CTA changes expert, and reloads
-        // its h fragments, once or twice.
+        // Down tickets: G contiguous ranges of equal cost over the shared and
+        // routed down units (shared tiles cost 2 stages, routed ones dn_stages),
+        // so a CTA changes expert, and reloads its h fragments, once or twice.
         constexpr int kDst = dn_stages<WF>();
         const long long cost = 2ll * usd + (long long)n * dn_tiles<WF>() * kDst;
         auto first = [&](long long cst) {
@@ -587,27 +588,30 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
 
     // ------------------------------ epilogue ------------------------------
     if (warp == kEpilogue) {
-        grid_dep_wait();
-        // per-expert tables, same ascending order as the producer's list
-        const int n = active_experts(a.offsets, a.E, lane, [&](int sg, int, int r0, int r1) {
-            if (sg < kMaxSeg) {
-                s.ep_rbase[sg] = r0;
-                s.ep_cnt[sg] = (uint8_t)(r1 - r0);
-            }
-        });
-        if (n > kMaxSeg) {
-            if (lane == 0) fail(a, s);
-            return;
-        }
-        __syncwarp();
-        for (int sg = lane; sg < n; sg += 32) {
-            const int rb = s.ep_rbase[sg], cnt = s.ep_cnt[sg];
+        // The shared gate/up units come first and need no routing; the
+        // per-expert tables (same ascending order as the producer's list) are
+        // built when the first other unit arrives.
+        int n = -1;
+        auto tables = [&]() {
+            grid_dep_wait();
+            n = active_experts(a.offsets, a.E, lane, [&](int sg, int, int r0, int r1) {
+                if (sg < kMaxSeg) {
+                    s.ep_rbase[sg] = r0;
+                    s.ep_cnt[sg] = (uint8_t)(r1 - r0);
+                }
+            });
+            if (n > kMaxSeg) return false;
+            __syncwarp();
+            for (int sg = lane; sg < n; sg += 32) {
+                const int rb = s.ep_rbase[sg], cnt = s.ep_cnt[sg];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (i < cnt) s.ep_tok[sg][i] = (uint8_t)(__ldcg(&a.perm[rb + i]) / a.k);
-        }
-        if (lane < a.T) s.ep_xs[lane] = a.xscale[lane].x;
-        __syncwarp();
+                for (int i = 0; i < 8; ++i)
+                    if (i < cnt) s.ep_tok[sg][i] = (uint8_t)(__ldcg(&a.perm[rb + i]) / a.k);
+            }
+            if (lane < a.T) s.ep_xs[lane] = a.xscale[lane].x;
+            __syncwarp();
+            return true;
+        };
         // gate/up tiles finished here and not yet published: shared, and routed of segment pseg
         uint32_t sh_fin = 0, r_fin = 0;
         int pseg = -1;
@@ -628,10 +632,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             if (!mbar_wait(&s.rfull[rb], (ru >> 1) & 1, &s.abort)) { fail(a, s); return; }
             const int m = s.rmeta[rb];
             if (m == -1) return;
-            if (m == -2) {  // before this CTA's first down unit: publish everything
+            if (m == -2) {  // before this CTA's first down unit (or its end): publish everything
                 publish();
                 if (lane == 0) mbar_arrive(&s.rempty[rb]);
                 continue;
+            }
+            if ((m >> 3) >= usg && n < 0 && !tables()) {
+                if (lane == 0) fail(a, s);
+                return;
             }
             const Unit un = unit_of<WF>(m >> 3, usg, n, usd);
             // Sum over the consumer warps of one column: lane l takes matrix
@@ -661,6 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                         if (lane < 16) a.hs[(int64_t)c * a.Fs + col] = f32_to_bf16_rne(silu_f32(v) * up);
                     }
                     ++sh_fin;
+                    publish();  // at once (one atomic per shared tile): nothing later waits on it
                 } else {
                     const int rbase = s.ep_rbase[un.seg], cnt = s.ep_cnt[un.seg];
                     for (int i = 0; i < cnt; ++i) {  // the expert's rows; column = the row's token
@@ -726,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     uint32_t Bm[4];             // Q2_K: sub-block sums (hi, lo)
     int bkind = -1, bseg = -2;  // what B holds
     bool dep = false;           // grid dependency resolved for this thread
-    bool flushed = false;       // gate/up count of this CTA published
+    bool flushed = false;       // gate/up counts of this CTA published
     float acc[2][4];
     int ru = 0;
     // Shared-memory addresses that stay fixed over stages. MXFP4 code words of
@@ -775,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             return;
         }
         const Unit un = unpack_unit(s.meta_k[slot]);
-        if (un.kind != kGsh && !dep) {
+        if (un.kind != kGsh && !dep) {  // the shared gate/up units need no routing
             grid_dep_wait();
             dep = true;
         }
@@ -785,6 +794,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             bkind = un.kind;
             bseg = useg;
             if (un.kind == kDsh || un.kind == kDrt) {  // every gate/up unit must be complete
+                // before the first down unit, this CTA's own gate/up counts go out
+                // (they all precede it in claim order)
                 if (!flushed) {
                     if (!marker(-2)) { fail(a, s); return; }
                     flushed = true;

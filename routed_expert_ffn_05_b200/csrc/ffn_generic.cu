@@ -7,7 +7,8 @@
 // experts are block-quantised, the shared expert is bf16 ("DS4", dibi8.com,
 // "Key architectural innovations" item 1; "DwarfStar", hysenlabs.com, "Model
 // support and quantisation"). In bf16-activation mode h is rounded to bf16
-// before W2; in MXFP8 mode x and h are quantised to MXFP8 along their length.
+// before W2; in MXFP8 (MXFP4) mode x and h are quantised to MXFP8 (MXFP4)
+// along their length.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -15,14 +16,16 @@
 
 namespace moe {
 
-struct ActRow {  // one activation row: bf16, fp32 (bf16-valued) or MXFP8
+struct ActRow {  // one activation row: bf16, fp32 (bf16-valued), MXFP8 or MXFP4
     const uint16_t *bf;
     const float *f;
-    const uint8_t *codes;
+    const uint8_t *codes;   // E4M3, one per byte
     const uint8_t *scales;
+    const uint8_t *codes4;  // E2M1, two per byte (element 2i in the low nibble)
     __device__ __forceinline__ float operator()(int i) const {
         if (bf) return bf16_to_f32(bf[i]);
         if (f) return f[i];
+        if (codes4) return e2m1_to_f32((codes4[i / 2] >> (4 * (i & 1))) & 15u) * e8m0_to_f32(scales[i / 32]);
         const __half_raw h = __nv_cvt_fp8_to_halfraw(codes[i], __NV_E4M3);
         return __half2float(__half(h)) * e8m0_to_f32(scales[i / 32]);
     }
@@ -85,8 +88,9 @@ __global__ void __launch_bounds__(256) gateup_generic_kernel(moe_dims d, MatRef 
     const int e = expert_of_row(offsets, d.E, r);
     const int t = perm[r] / d.k;
     const int K = d.d_model;
-    ActRow a{nullptr, nullptr, nullptr, nullptr};
+    ActRow a{nullptr, nullptr, nullptr, nullptr, nullptr};
     if (d.act == MOE_A_MXFP8) { a.codes = x8 + (int64_t)t * K; a.scales = xs + (int64_t)t * (K / 32); }
+    else if (d.act == MOE_A_MXFP4) { a.codes4 = x8 + (int64_t)t * (K / 2); a.scales = xs + (int64_t)t * (K / 32); }
     else a.bf = x + (int64_t)t * K;
     const int64_t row = (int64_t)e * d.d_ff + n;
     float g = 0.0f, u = 0.0f;
@@ -112,8 +116,9 @@ __global__ void __launch_bounds__(256) down_generic_kernel(moe_dims d, MatRef w2
     if (i >= d.d_model) return;
     const int e = expert_of_row(offsets, d.E, r);
     const int K = d.d_ff;
-    ActRow a{nullptr, nullptr, nullptr, nullptr};
+    ActRow a{nullptr, nullptr, nullptr, nullptr, nullptr};
     if (d.act == MOE_A_MXFP8) { a.codes = h8 + (int64_t)r * K; a.scales = hs + (int64_t)r * (K / 32); }
+    else if (d.act == MOE_A_MXFP4) { a.codes4 = h8 + (int64_t)r * (K / 2); a.scales = hs + (int64_t)r * (K / 32); }
     else a.f = h + (int64_t)r * K;
     const int64_t row = (int64_t)e * d.d_model + i;
     float o = 0.0f;
@@ -130,12 +135,11 @@ cudaError_t launch_expert_ffn_generic(const moe_dims &d, const moe_weights &w, c
     uint8_t *x8 = ws + L.x8, *xs = ws + L.xs, *h8 = ws + L.h8, *hs = ws + L.hs;
     float *h = reinterpret_cast<float *>(ws + L.h);
     cudaError_t err;
-    if (d.act == MOE_A_MXFP8 && (err = launch_quant_act_bf16(x, d.T, d.d_model, x8, xs, s)) != cudaSuccess)
-        return err;
+    const bool q = d.act != MOE_A_BF16, fp4 = d.act == MOE_A_MXFP4;
+    if (q && (err = launch_quant_act_bf16(x, d.T, d.d_model, x8, xs, s, fp4)) != cudaSuccess) return err;
     gateup_generic_kernel<<<dim3((unsigned)S, ceil_div(d.d_ff, 8)), 256, 0, s>>>(
         d, mat_ref(d, MOE_MAT_W1, w.w1), mat_ref(d, MOE_MAT_W3, w.w3), x, x8, xs, offsets, perm, h);
-    if (d.act == MOE_A_MXFP8 && (err = launch_quant_act_f32(h, S, d.d_ff, h8, hs, s)) != cudaSuccess)
-        return err;
+    if (q && (err = launch_quant_act_f32(h, S, d.d_ff, h8, hs, s, fp4)) != cudaSuccess) return err;
     down_generic_kernel<<<dim3((unsigned)S, ceil_div(d.d_model, 8)), 256, 0, s>>>(
         d, mat_ref(d, MOE_MAT_W2, w.w2), h, h8, hs, offsets, out_rows);
     count_launches(2);
@@ -195,6 +199,7 @@ cudaError_t launch_expert_ffn(const moe_dims &d, const moe_weights &w, const uin
         (e = launch_shared_ffn_generic(d, w, x, shared_out, reinterpret_cast<float *>(ws + L.sh_h), s)) != cudaSuccess)
         return e;
     if (tc_path_applies(d)) return launch_tc_ffn(d, w, x, offsets, perm, out_rows, ws, L, s, rows_bf16);
+    if (tc16_path_applies(d)) return launch_tc16_ffn(d, w, x, offsets, perm, out_rows, ws, L, s);
     return launch_expert_ffn_generic(d, w, x, offsets, perm, out_rows, ws, L, s);
 }
 

@@ -58,10 +58,12 @@ cudaError_t launch_pack_weights(const moe_dims &d, int which, const uint8_t *can
                                 cudaStream_t s);
 cudaError_t launch_debug_dequant(const moe_dims &d, int which, const uint8_t *packed, int expert,
                                  float *out, cudaStream_t s);
+// MX quantisation of activation rows: MXFP8 codes [rows][K], or MXFP4 (fp4)
+// codes [rows][K/2]; E8M0 scales [rows][K/32].
 cudaError_t launch_quant_act_bf16(const uint16_t *x, int64_t rows, int K, uint8_t *codes, uint8_t *scales,
-                                  cudaStream_t s);
+                                  cudaStream_t s, bool fp4 = false);
 cudaError_t launch_quant_act_f32(const float *x, int64_t rows, int K, uint8_t *codes, uint8_t *scales,
-                                 cudaStream_t s);
+                                 cudaStream_t s, bool fp4 = false);
 
 // Routed expert FFN over all permuted rows (ws gives h / h8 / x8 scratch), and
 // the shared expert into `shared_out` when it is non-null.
@@ -95,6 +97,16 @@ bool tc_path_applies(const moe_dims &d);
 cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
                           const int32_t *perm, float *out_rows, uint8_t *ws, const WsLayout &L, cudaStream_t s,
                           bool rows_bf16 = false);
+
+// Token-tile plan (ustart [E+1]) and the slot -> row inverse of perm (row_of [S], -1 for slots without a row).
+cudaError_t launch_tc_plan(const moe_dims &d, const int32_t *offsets, const int32_t *perm, int32_t *ustart,
+                           int32_t *row_of, cudaStream_t s);
+
+// w4a16 (bf16 activations, MXFP4 weights) on the tensor cores, batches the
+// decode path does not take.
+bool tc16_path_applies(const moe_dims &d);
+cudaError_t launch_tc16_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
+                            const int32_t *perm, float *out_rows, uint8_t *ws, const WsLayout &L, cudaStream_t s);
 
 // The tensor-core path's activation staging alone (also a test hook).
 cudaError_t launch_tc_gather(const moe_dims &d, const uint16_t *x, const int32_t *offsets, const int32_t *perm,

@@ -66,7 +66,7 @@ struct TcArgs {
 struct TcSmem {
     uint8_t a[kTcStages][2][kTileBytes];
     uint8_t b[kTcStages][kTileBytes];
-    uint8_t sf[kTcStages][3][512];
+    uint8_t sf[kTcStages][3][1024];  // E8M0 atoms per stage: W (rows 0..127), W (128..255), tokens
     uint64_t full[kTcStages], empty[kTcStages], acc_full, acc_empty, mma_done;
     uint32_t tmem_base;
     volatile int abort;
@@ -119,6 +119,20 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
     return r;
 }
 
+// Eight fp32 values times sc -> eight E2M1 codes in one word (element i in
+// bits 4i .. 4i + 3), round to nearest even, saturating (hardware conversion).
+__device__ __forceinline__ uint32_t e2m1x8(const float *v, float sc) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t b;
+        asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+            : "=r"(b) : "f"(v[2 * i + 1] * sc), "f"(v[2 * i] * sc));
+        w |= b << (8 * i);
+    }
+    return w;
+}
+
 // Two fp32 -> bf16 (round to nearest even), the first in the low half.
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
     return (uint32_t)f32_to_bf16_rne(lo) | (uint32_t)f32_to_bf16_rne(hi) << 16;
@@ -127,15 +141,23 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
 // 2^-se as an fp32 (exact for se in [-127, 126]).
 __device__ __forceinline__ float pow2_neg(int se) { return __uint_as_float((uint32_t)(127 - se) << 23); }
 
-template <int MODE>
+// AF: the activations' element bits. 8: E4M3 tokens against E2M1 weights on
+// kind::mxf8f6f4 (the weights expanded to a byte per element by the tensor
+// map; one 128-byte row of a box is K = 128, one MMA is K = 32). 4: E2M1 on
+// both sides on kind::mxf4 (packed two per byte; a box row is K = 256, one
+// MMA is K = 64 with two E8M0 scales per row, scale_vec::2X).
+template <int MODE, int AF>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     TcSmem &s = tc_smem(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool GU = MODE == kModeGU;
+    constexpr int kKs = AF == 8 ? kTile : 2 * kTile;   // K per stage
+    constexpr int kAt = kKs / 128;                     // E8M0 atoms (128 rows x 128 K) per operand per stage
+    constexpr int kSfStage = AF == 8 ? 16 : 24;        // TMEM scale columns per stage
     // work items per expert and token tile: 128 gate+up rows (gate/up) or 256
     // down rows (down), both as two 128-row MMA operands per K step
-    const int ft = a.Nw / (GU ? kTile : 2 * kTile), kt_n = a.K / kTile;
+    const int ft = a.Nw / (GU ? kTile : 2 * kTile), kt_n = a.K / kKs, at_n = a.K / 128;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTcStages; ++i) {
@@ -165,27 +187,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             prefetch_tensormap(&a.wa);
             prefetch_tensormap(&a.act);
             // an expanded E2M1 box credits the packed bytes it reads (8 KB), not
-            // the 16 KB it fills in shared memory
-            const uint32_t tx = 2 * (kTileBytes / 2) + kTileBytes + 3 * 512;
+            // the 16 KB it fills in shared memory; packed boxes credit 16 KB
+            const uint32_t tx = (AF == 8 ? kTileBytes : 2 * kTileBytes) + kTileBytes + 3 * 512 * kAt;
             int it = 0;
             for (int w = blockIdx.x; w < n_work && !s.abort; w += gridDim.x) {
                 const Work wk = work_of(w, ft, s.ustart, a.E, a.offsets);
                 // the two weight tiles: W1 and W3 rows 128 f (gate/up), W2 rows 256 f and 256 f + 128 (down)
                 const int wrow0 = wk.e * a.Nw + wk.f * (GU ? kTile : 2 * kTile), wrow1 = GU ? wrow0 : wrow0 + kTile;
                 const int64_t rg0 = (int64_t)wk.e * (a.Nw / kTile) + (GU ? wk.f : 2 * wk.f);  // 128-row group
-                const int64_t wat0 = rg0 * kt_n, wat1 = (GU ? rg0 : rg0 + 1) * kt_n;        // weight atom bases
-                const int64_t aat = ((int64_t)s.ustart[wk.e] + wk.j) * kt_n;              // activation atom base
+                const int64_t wat0 = rg0 * at_n, wat1 = (GU ? rg0 : rg0 + 1) * at_n;        // weight atom bases
+                const int64_t aat = ((int64_t)s.ustart[wk.e] + wk.j) * at_n;              // activation atom base
                 for (int kt = 0; kt < kt_n; ++kt, ++it) {
                     const int slot = it % kTcStages;
                     if (!mbar_wait(&s.empty[slot], ((it / kTcStages) & 1) ^ 1)) { tc_fail(a, s); break; }
                     uint64_t *bar = &s.full[slot];
                     mbar_arrive_expect_tx(bar, tx);
+                    // box x coordinate: 128 K-elements (AF 8, expanded map) or 128 bytes = 256 K (AF 4)
                     tma_load_2d(s.a[slot][0], &a.wa, kt * kTile, wrow0, bar);
                     tma_load_2d(s.a[slot][1], &a.wb, kt * kTile, wrow1, bar);
                     tma_load_2d(s.b[slot], &a.act, kt * kTile, wk.row0, bar);
-                    bulk_g2s(s.sf[slot][0], a.sfa + (wat0 + kt) * 512, 512, bar);
-                    bulk_g2s(s.sf[slot][1], a.sfb + (wat1 + kt) * 512, 512, bar);
-                    bulk_g2s(s.sf[slot][2], a.sfact + (aat + kt) * 512, 512, bar);
+                    bulk_g2s(s.sf[slot][0], a.sfa + (wat0 + kAt * kt) * 512, 512 * kAt, bar);
+                    bulk_g2s(s.sf[slot][1], a.sfb + (wat1 + kAt * kt) * 512, 512 * kAt, bar);
+                    bulk_g2s(s.sf[slot][2], a.sfact + (aat + kAt * kt) * 512, 512 * kAt, bar);
                 }
             }
             // copies in flight land before the CTA exits
@@ -197,10 +220,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         if (lane == 0) {
             int it = 0, lw = 0;
             for (int w = blockIdx.x; w < n_work && !s.abort; w += gridDim.x, ++lw) {
-                // A = the token tile (E4M3, M = 128), B = both 128-row weight tiles
-                // as one 256-row operand (E2M1, N = 256): one MMA per K step
-                // yields gate and up (or 256 down features) for every token
-                constexpr uint32_t idesc = idesc_mx(0, 5, 128, 256);
+                // A = the token tile (E4M3 or E2M1, M = 128), B = both 128-row
+                // weight tiles as one 256-row operand (E2M1, N = 256): one MMA per
+                // K step yields gate and up (or 256 down features) for every token
+                // (format codes: mxf8f6f4 E4M3 0, E2M1 5; mxf4 E2M1 1)
+                constexpr uint32_t idesc = AF == 8 ? idesc_mx(0, 5, 128, 256) : idesc_mx(1, 1, 128, 256);
                 if (!mbar_wait(&s.acc_empty, (lw & 1) ^ 1)) { tc_fail(a, s); break; }
                 tc_fence_after();
                 bool ok = true;
@@ -208,18 +232,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                     const int slot = it % kTcStages;
                     if (!mbar_wait(&s.full[slot], (it / kTcStages) & 1)) { ok = false; break; }
                     tc_fence_after();
-                    // scale columns: weight rows 0..127 at +0, 128..255 at +4 (B reads
-                    // column n / 32), tokens at +8 (A reads column m / 32)
-                    const uint32_t sfc = tmem + kSfCol + 16 * slot;
-                    tc_cp_sf(sfc, sdesc_sf(s.sf[slot][0]));
-                    tc_cp_sf(sfc + 4, sdesc_sf(s.sf[slot][1]));
-                    tc_cp_sf(sfc + 8, sdesc_sf(s.sf[slot][2]));
+                    // scale columns of atom at (K 128 at .. + 127): weight rows 0..127 at
+                    // +8 at, 128..255 at +8 at + 4 (B reads column n / 32), tokens at
+                    // +8 kAt + 4 at (A reads column m / 32); a column's byte j is 32-block j
+                    const uint32_t sfc = tmem + kSfCol + kSfStage * slot;
+#pragma unroll
+                    for (int at = 0; at < kAt; ++at) {
+                        tc_cp_sf(sfc + 8 * at, sdesc_sf(s.sf[slot][0] + 512 * at));
+                        tc_cp_sf(sfc + 8 * at + 4, sdesc_sf(s.sf[slot][1] + 512 * at));
+                        tc_cp_sf(sfc + 8 * kAt + 4 * at, sdesc_sf(s.sf[slot][2] + 512 * at));
+                    }
                     const uint64_t dt = sdesc_sw128(s.b[slot]), dw = sdesc_sw128(s.a[slot][0]);  // a[slot][0..1]: 256 rows
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint32_t id = idesc_sf_ids(idesc, ks, ks), acc = (kt | ks) != 0;
-                        const uint32_t sel = (uint32_t)ks << 30;
-                        tc_mma_mx(tmem, dt + 2 * ks, dw + 2 * ks, id, (sfc + 8) | sel, sfc | sel, acc);
+                    for (int ks = 0; ks < 4; ++ks) {  // 32 bytes of every row per MMA
+                        const uint32_t acc = (kt | ks) != 0;
+                        if (AF == 8) {  // K 32: one scale per row, byte ks of the stage's atom
+                            const uint32_t id = idesc_sf_ids(idesc, ks, ks), sel = (uint32_t)ks << 30;
+                            tc_mma_mx(tmem, dt + 2 * ks, dw + 2 * ks, id, (sfc + 8) | sel, sfc | sel, acc);
+                        } else {        // K 64: scales 2 (ks % 2), + 1 of atom ks / 2
+                            const uint32_t b0 = 2 * (ks & 1), at = ks >> 1;
+                            const uint32_t id = idesc_sf_ids(idesc, b0, b0), sel = b0 << 30;
+                            tc_mma_mxf4(tmem, dt + 2 * ks, dw + 2 * ks, id, (sfc + 8 * kAt + 4 * at) | sel,
+                                        (sfc + 8 * at) | sel, acc);
+                        }
                     }
                     tc_commit(&s.empty[slot]);  // frees the stage once these MMAs finish
                 }
@@ -297,9 +332,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                     v[i] = __uint_as_float(g0[i]);
                     v[32 + i] = __uint_as_float(g1[i]);
                 }
-                // MXFP8 along F: each block of 32 is 32 of this thread's values
+                // MXFP8 (MXFP4) along F: each block of 32 is 32 of this thread's
+                // values; scale 2^(floor(log2 amax) - 8 (2)), an all-zero block
+                // gets scale byte 127 (and codes of +-0)
                 const int64_t atom = (((int64_t)s.ustart[wk.e] + wk.j) * (a.Nw / kTile) + wk.f) * 512;
-                uint8_t *hrow = a.h8 + (int64_t)(wk.row0 + t) * a.Nw + wk.f * kTile + 64 * half;
+                uint8_t *hrow = a.h8 + (int64_t)(wk.row0 + t) * (a.Nw * AF / 8) + (wk.f * kTile + 64 * half) * AF / 8;
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
                     uint32_t amax = 0;
@@ -308,21 +345,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
                     int se = 0;
                     float sc = 0.0f;
                     if (amax != 0u) {
-                        const int e8 = floor_log2_f32(__uint_as_float(amax)) - 8;
-                        se = e8 < -127 ? -127 : (e8 > 127 ? 127 : e8);
+                        const int ee = floor_log2_f32(__uint_as_float(amax)) - (AF == 8 ? 8 : 2);
+                        se = ee < -127 ? -127 : (ee > 127 ? 127 : ee);
                         sc = pow2_neg(se);
                     }
-                    uint32_t pk[8];
+                    if (AF == 8) {
+                        uint32_t pk[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        pk[i] = f32x2_to_e4m3x2(v[32 * bb + 4 * i] * sc, v[32 * bb + 4 * i + 1] * sc) |
-                                f32x2_to_e4m3x2(v[32 * bb + 4 * i + 2] * sc, v[32 * bb + 4 * i + 3] * sc) << 16;
-                    if (valid) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(hrow + 32 * bb);
-                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                        a.hsf[atom + sf_atom_byte(t, 2 * half + bb)] = (uint8_t)(se + 127);
+                        for (int i = 0; i < 8; ++i)
+                            pk[i] = f32x2_to_e4m3x2(v[32 * bb + 4 * i] * sc, v[32 * bb + 4 * i + 1] * sc) |
+                                    f32x2_to_e4m3x2(v[32 * bb + 4 * i + 2] * sc, v[32 * bb + 4 * i + 3] * sc) << 16;
+                        if (valid) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(hrow + 32 * bb);
+                            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        }
+                    } else {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            pk[i] = e2m1x8(&v[32 * bb + 8 * i], sc);
+                        if (valid) *reinterpret_cast<uint4 *>(hrow + 16 * bb) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
+                    if (valid) a.hsf[atom + sf_atom_byte(t, 2 * half + bb)] = (uint8_t)(se + 127);
                 }
             } else if (valid) {
                 const int64_t o0 = (int64_t)(wk.row0 + t) * a.Nw + wk.f * 2 * kTile + 128 * half;
@@ -394,11 +439,13 @@ __global__ void __launch_bounds__(1024) tc_plan_kernel(const int32_t *__restrict
     if (e == E - 1) ustart[E] = excl + nt;
 }
 
-// One warp per token: its x row becomes MXFP8 once (E4M3 codes and E8M0
-// scales per 32 along d, the OCP rule: scale exponent floor(log2 amax) - 8,
-// RNE, saturating; an all-zero block gets scale 127 and zero codes), and the
-// codes go to each of the token's k rows in expert order, the scales to those
-// rows' token-tile atoms. x is read once per token instead of once per row.
+// One warp per token: its x row becomes MXFP8 (AF 8: E4M3 codes) or MXFP4
+// (AF 4: E2M1 codes, two per byte) once, with E8M0 scales per 32 along d (the
+// OCP rule: scale exponent floor(log2 amax) - 8 or - 2, RNE, saturating; an
+// all-zero block gets scale 127 and zero codes), and the codes go to each of
+// the token's k rows in expert order, the scales to those rows' token-tile
+// atoms. x is read once per token instead of once per row.
+template <int AF>
 __global__ void __launch_bounds__(256) tc_gather_quant_kernel(const uint16_t *__restrict__ x,
                                                               const int32_t *__restrict__ offsets,
                                                               const int32_t *__restrict__ row_of,
@@ -450,19 +497,24 @@ __global__ void __launch_bounds__(256) tc_gather_quant_kernel(const uint16_t *__
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
             uint32_t lo = 0, hi = 0, sb = 127;
             if (amax > 0.0f) {
-                int se = floor_log2_f32(amax) - 8;
+                int se = floor_log2_f32(amax) - (AF == 8 ? 8 : 2);
                 se = se < -127 ? -127 : (se > 127 ? 127 : se);
                 sb = (uint32_t)(se + 127);
                 const float sc = pow2_neg(se);
-                lo = f32x2_to_e4m3x2(f[0] * sc, f[1] * sc) | f32x2_to_e4m3x2(f[2] * sc, f[3] * sc) << 16;
-                hi = f32x2_to_e4m3x2(f[4] * sc, f[5] * sc) | f32x2_to_e4m3x2(f[6] * sc, f[7] * sc) << 16;
+                if (AF == 8) {
+                    lo = f32x2_to_e4m3x2(f[0] * sc, f[1] * sc) | f32x2_to_e4m3x2(f[2] * sc, f[3] * sc) << 16;
+                    hi = f32x2_to_e4m3x2(f[4] * sc, f[5] * sc) | f32x2_to_e4m3x2(f[6] * sc, f[7] * sc) << 16;
+                } else {
+                    lo = e2m1x8(f, sc);
+                }
             }
             if (i0 >= d) continue;
             const int b = i0 / 32;
             for (int j = 0; j < k; ++j) {
                 const int row = s_row[wl][j];
                 if (row < 0) continue;
-                *reinterpret_cast<uint2 *>(x8 + (int64_t)row * d + i0) = make_uint2(lo, hi);
+                if (AF == 8) *reinterpret_cast<uint2 *>(x8 + (int64_t)row * d + i0) = make_uint2(lo, hi);
+                else *reinterpret_cast<uint32_t *>(x8 + (int64_t)row * (d / 2) + i0 / 2) = lo;
                 if ((lane & 3) == 0) xsf[(s_atom[wl][j] + b / 4) * 512 + sf_atom_byte(s_rt[wl][j], b % 4)] = (uint8_t)sb;
             }
         }
@@ -481,10 +533,10 @@ cudaError_t tc_set_attrs() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(tc_ffn_kernel<kModeGU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)))
-        return e;
-    if ((e = cudaFuncSetAttribute(tc_ffn_kernel<kModeDN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes)))
-        return e;
+    void (*const kernels[4])(TcArgs) = {tc_ffn_kernel<kModeGU, 8>, tc_ffn_kernel<kModeDN, 8>,
+                                        tc_ffn_kernel<kModeGU, 4>, tc_ffn_kernel<kModeDN, 4>};
+    for (auto k : kernels)
+        if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes))) return e;
     done[dev].store(true, std::memory_order_release);
     return cudaSuccess;
 }
@@ -492,12 +544,15 @@ cudaError_t tc_set_attrs() {
 }  // namespace
 
 bool tc_path_applies(const moe_dims &d) {
-    return d.wfmt == MOE_W_MXFP4 && d.act == MOE_A_MXFP8 && d.d_model % (2 * kTile) == 0 && d.d_ff % kTile == 0 &&
-           d.E <= kTcMaxE && d.T >= 1;
+    // K per stage: 128 (w4a8) or 256 (w4a4) for both GEMMs (K = d_model, d_ff)
+    const int ks = d.act == MOE_A_MXFP4 ? 2 * kTile : kTile;
+    return d.wfmt == MOE_W_MXFP4 && (d.act == MOE_A_MXFP8 || d.act == MOE_A_MXFP4) && d.d_model % (2 * kTile) == 0 &&
+           d.d_model % ks == 0 && d.d_ff % ks == 0 && d.E <= kTcMaxE && d.T >= 1;
 }
 
-// Routed expert FFN (w4a8, MXFP4 weights) on the tensor cores: plan, gather +
-// quantise, gate/up GEMM with SwiGLU and MXFP8 requantisation, down GEMM.
+// Routed expert FFN (MXFP4 weights; w4a8 or w4a4) on the tensor cores: plan,
+// gather + quantise, gate/up GEMM with SwiGLU and MXFP8 (MXFP4)
+// requantisation, down GEMM.
 cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_t *x, const int32_t *offsets,
                           const int32_t *perm, float *out_rows, uint8_t *ws, const WsLayout &L, cudaStream_t s,
                           bool rows_bf16) {
@@ -513,15 +568,25 @@ cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_
 
     TcArgs g;
     memset(&g, 0, sizeof g);
-    const uint64_t r13 = (uint64_t)d.E * d.d_ff, r2 = (uint64_t)d.E * d.d_model;
-    bool ok = make_tile_map_e2m1(&g.wa, p1 + L1.codes, r13, d.d_model, kTile) &&
-              make_tile_map_e2m1(&g.wb, p3 + L1.codes, r13, d.d_model, kTile) &&
-              make_tile_map_u8(&g.act, gx8, S, d.d_model, kTile);
     TcArgs dn;
     memset(&dn, 0, sizeof dn);
-    ok = ok && make_tile_map_e2m1(&dn.wa, p2 + L2.codes, r2, d.d_ff, kTile) &&
-         make_tile_map_e2m1(&dn.wb, p2 + L2.codes, r2, d.d_ff, kTile) &&
-         make_tile_map_u8(&dn.act, h8, S, d.d_ff, kTile);
+    const uint64_t r13 = (uint64_t)d.E * d.d_ff, r2 = (uint64_t)d.E * d.d_model;
+    const bool a4 = d.act == MOE_A_MXFP4;
+    bool ok;
+    if (a4)  // packed E2M1 on both sides: byte boxes of 128 x 128
+        ok = make_tile_map_u8(&g.wa, p1 + L1.codes, r13, d.d_model / 2, kTile) &&
+             make_tile_map_u8(&g.wb, p3 + L1.codes, r13, d.d_model / 2, kTile) &&
+             make_tile_map_u8(&g.act, gx8, S, d.d_model / 2, kTile) &&
+             make_tile_map_u8(&dn.wa, p2 + L2.codes, r2, d.d_ff / 2, kTile) &&
+             make_tile_map_u8(&dn.wb, p2 + L2.codes, r2, d.d_ff / 2, kTile) &&
+             make_tile_map_u8(&dn.act, h8, S, d.d_ff / 2, kTile);
+    else     // E2M1 weights expanded to a byte per element beside E4M3 tokens
+        ok = make_tile_map_e2m1(&g.wa, p1 + L1.codes, r13, d.d_model, kTile) &&
+             make_tile_map_e2m1(&g.wb, p3 + L1.codes, r13, d.d_model, kTile) &&
+             make_tile_map_u8(&g.act, gx8, S, d.d_model, kTile) &&
+             make_tile_map_e2m1(&dn.wa, p2 + L2.codes, r2, d.d_ff, kTile) &&
+             make_tile_map_e2m1(&dn.wb, p2 + L2.codes, r2, d.d_ff, kTile) &&
+             make_tile_map_u8(&dn.act, h8, S, d.d_ff, kTile);
     if (!ok) return cudaErrorInvalidValue;
     g.sfa = p1 + L1.stile; g.sfb = p3 + L1.stile; g.sfact = gxsf;
     g.offsets = offsets; g.ustart = ustart; g.E = d.E; g.Nw = d.d_ff; g.K = d.d_model;
@@ -535,26 +600,45 @@ cudaError_t launch_tc_ffn(const moe_dims &d, const moe_weights &w, const uint16_
     if ((e = launch_tc_gather(d, x, offsets, perm, ustart, reinterpret_cast<int32_t *>(ws + L.row_of), gx8, gxsf, s)))
         return e;
     const int grid = tc_num_sms();
-    tc_ffn_kernel<kModeGU><<<grid, kTcThreads, kTcSmemBytes, s>>>(g);
-    tc_ffn_kernel<kModeDN><<<grid, kTcThreads, kTcSmemBytes, s>>>(dn);
+    if (a4) {
+        tc_ffn_kernel<kModeGU, 4><<<grid, kTcThreads, kTcSmemBytes, s>>>(g);
+        tc_ffn_kernel<kModeDN, 4><<<grid, kTcThreads, kTcSmemBytes, s>>>(dn);
+    } else {
+        tc_ffn_kernel<kModeGU, 8><<<grid, kTcThreads, kTcSmemBytes, s>>>(g);
+        tc_ffn_kernel<kModeDN, 8><<<grid, kTcThreads, kTcSmemBytes, s>>>(dn);
+    }
     count_launches(2);
     return cudaGetLastError();
 }
 
 // The tensor-core path's activation staging: token-tile plan, slot -> row
-// inverse of perm, and the MXFP8 rows in expert order with their scale atoms
-// (gx8 [S][d], gxsf [tiles][d/128][512], ustart [E+1]).
+// inverse of perm, and the MXFP8 (MXFP4) rows in expert order with their
+// scale atoms (gx8 [S][d] ([S][d/2]), gxsf [tiles][d/128][512], ustart [E+1]).
+cudaError_t launch_tc_plan(const moe_dims &d, const int32_t *offsets, const int32_t *perm, int32_t *ustart,
+                           int32_t *row_of, cudaStream_t s) {
+    const int S = d.T * d.k;
+    if (S == 0) return cudaSuccess;
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(row_of, 0xFF, (size_t)S * 4, s)) != cudaSuccess) return e;
+    tc_plan_kernel<<<1 + (S + 1023) / 1024, 1024, 0, s>>>(offsets, d.E, ustart, perm, S, row_of, device_error_word());
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_tc_gather(const moe_dims &d, const uint16_t *x, const int32_t *offsets, const int32_t *perm,
                              int32_t *ustart, int32_t *row_of, uint8_t *gx8, uint8_t *gxsf, cudaStream_t s) {
     const int S = d.T * d.k;
     if (S == 0) return cudaSuccess;
     cudaError_t e;
     int *err = device_error_word();
-    if ((e = cudaMemsetAsync(row_of, 0xFF, (size_t)S * 4, s)) != cudaSuccess) return e;
-    tc_plan_kernel<<<1 + (S + 1023) / 1024, 1024, 0, s>>>(offsets, d.E, ustart, perm, S, row_of, err);
-    tc_gather_quant_kernel<<<(d.T + 7) / 8, 256, 0, s>>>(x, offsets, row_of, ustart, d.T, d.E, d.k, d.d_model, gx8,
-                                                         gxsf, err);
-    count_launches(2);
+    if ((e = launch_tc_plan(d, offsets, perm, ustart, row_of, s)) != cudaSuccess) return e;
+    if (d.act == MOE_A_MXFP4)
+        tc_gather_quant_kernel<4><<<(d.T + 7) / 8, 256, 0, s>>>(x, offsets, row_of, ustart, d.T, d.E, d.k, d.d_model,
+                                                                gx8, gxsf, err);
+    else
+        tc_gather_quant_kernel<8><<<(d.T + 7) / 8, 256, 0, s>>>(x, offsets, row_of, ustart, d.T, d.E, d.k, d.d_model,
+                                                                gx8, gxsf, err);
+    count_launches(1);
     return cudaGetLastError();
 }
 

@@ -72,6 +72,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     return true;
 }
 
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy ones (a TMA copy into the same bytes).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Global -> shared bulk copy (16-byte aligned, size a multiple of 16) that
 // completes `bytes` of transaction count on `bar`.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

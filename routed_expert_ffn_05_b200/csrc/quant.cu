@@ -227,7 +227,10 @@ __device__ __forceinline__ float load_act<uint16_t>(const uint16_t *p, int64_t i
 template <>
 __device__ __forceinline__ float load_act<float>(const float *p, int64_t i) { return p[i]; }
 
-template <typename T>
+// One thread per 32-element block: MXFP8 (AF 8, E4M3 codes [rows][K]) or
+// MXFP4 (AF 4, E2M1 codes [rows][K/2], element 2i in the low nibble), E8M0
+// scales [rows][K/32]; the OCP rule with emax 8 or 2.
+template <typename T, int AF>
 __global__ void quant_act_kernel(const T *__restrict__ x, int64_t rows, int K, uint8_t *__restrict__ codes,
                                  uint8_t *__restrict__ scales) {
     const int64_t nb = K / 32;
@@ -243,34 +246,46 @@ __global__ void quant_act_kernel(const T *__restrict__ x, int64_t rows, int K, u
     uint32_t packed[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     uint8_t sb = 127;
     if (amax > 0.0f) {
-        const int se = mx_shared_exp(amax, 8);
+        const int se = mx_shared_exp(amax, AF == 8 ? 8 : 2);
         sb = (uint8_t)(se + 127);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const uint32_t c = __nv_cvt_float_to_fp8(ldexpf(v[i], -se), __NV_SATFINITE, __NV_E4M3);
-            packed[i / 4] |= c << (8 * (i % 4));
+        for (int i = 0; i < 32; i += AF == 8 ? 1 : 2) {
+            if (AF == 8) {
+                const uint32_t c = __nv_cvt_float_to_fp8(ldexpf(v[i], -se), __NV_SATFINITE, __NV_E4M3);
+                packed[i / 4] |= c << (8 * (i % 4));
+            } else {
+                packed[i / 8] |= f32x2_to_e2m1x2(ldexpf(v[i], -se), ldexpf(v[i + 1], -se)) << (8 * ((i / 2) % 4));
+            }
         }
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(codes + base);
-    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    if (AF == 8) {
+        uint4 *dst = reinterpret_cast<uint4 *>(codes + base);
+        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    } else {
+        *reinterpret_cast<uint4 *>(codes + base / 2) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
     scales[blk] = sb;
 }
 
 cudaError_t launch_quant_act_bf16(const uint16_t *x, int64_t rows, int K, uint8_t *codes, uint8_t *scales,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, bool fp4) {
     const int64_t nb = rows * (K / 32);
     if (nb == 0) return cudaSuccess;
-    quant_act_kernel<uint16_t><<<(unsigned)((nb + 255) / 256), 256, 0, s>>>(x, rows, K, codes, scales);
+    const unsigned g = (unsigned)((nb + 255) / 256);
+    if (fp4) quant_act_kernel<uint16_t, 4><<<g, 256, 0, s>>>(x, rows, K, codes, scales);
+    else quant_act_kernel<uint16_t, 8><<<g, 256, 0, s>>>(x, rows, K, codes, scales);
     count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quant_act_f32(const float *x, int64_t rows, int K, uint8_t *codes, uint8_t *scales,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, bool fp4) {
     const int64_t nb = rows * (K / 32);
     if (nb == 0) return cudaSuccess;
-    quant_act_kernel<float><<<(unsigned)((nb + 255) / 256), 256, 0, s>>>(x, rows, K, codes, scales);
+    const unsigned g = (unsigned)((nb + 255) / 256);
+    if (fp4) quant_act_kernel<float, 4><<<g, 256, 0, s>>>(x, rows, K, codes, scales);
+    else quant_act_kernel<float, 8><<<g, 256, 0, s>>>(x, rows, K, codes, scales);
     count_launches(1);
     return cudaGetLastError();
 }

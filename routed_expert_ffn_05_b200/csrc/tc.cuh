@@ -54,6 +54,18 @@ __device__ __forceinline__ void tc_mma_mx(uint32_t d, uint64_t adesc, uint64_t b
         : "memory");
 }
 
+// The same for kind::mxf4: A and B packed E2M1 (two per byte), K = 64, two
+// E8M0 scale factors per row (scale_vec::2X: bytes sf id and sf id + 1 of the
+// TMEM scale word, sf id 0 or 2).
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                            uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
 // D[M][N] (+)= A[M][K] . B[N][K]^T with K = 16 bf16 elements, fp32 accumulate
 // in TMEM; A and B in shared memory (descriptors).
 __device__ __forceinline__ void tc_mma_bf16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -64,6 +76,31 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d, uint64_t adesc, uint64_t
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+
+// The same with A in tensor memory (lane m = row m of A, K-major, two bf16 per
+// 32-bit column: K = 16 is 8 columns from a_tmem); B from shared memory.
+__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Thread i of the warp writes TMEM lane (lane field of taddr) + i, columns
+// taddr .. taddr + 31, from r[0 .. 31].
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Thread i of the warp reads TMEM lane (lane field of taddr) + i, columns
 // taddr .. taddr + 31 (one 32-bit value per column).
@@ -99,9 +136,11 @@ __device__ __forceinline__ uint64_t sdesc_sf(const void *p) {
     return ((a >> 4) & 0x3FFFull) | (8ull << 32) | (1ull << 46);
 }
 
-// Instruction descriptor of kind::mxf8f6f4 with E8M0 scales, both operands
-// K-major, dense K = 32. Formats: 0 = E4M3, 5 = E2M1. The scale-factor byte
-// ids (which of the 4 bytes of each TMEM word) are or-ed in per K step.
+// Instruction descriptor of the block-scaled kinds with E8M0 scales (bit 23),
+// both operands K-major, dense K (32 for kind::mxf8f6f4, 64 for kind::mxf4:
+// bit 31 clear). Formats: mxf8f6f4 0 = E4M3, 5 = E2M1; mxf4 1 = E2M1. The
+// scale-factor byte ids (which of the 4 bytes of each TMEM word) are or-ed in
+// per K step.
 __host__ __device__ constexpr uint32_t idesc_mx(int a_fmt, int b_fmt, int M, int N) {
     return (uint32_t)(a_fmt & 7) << 7 | (uint32_t)(b_fmt & 7) << 10 | (uint32_t)(N >> 3) << 17 | 1u << 23 |
            (uint32_t)(M >> 4) << 24;

@@ -85,7 +85,7 @@ class Case:
         self.ora = self.hw.oracle_layer(cfg, self.wr, self.bias, self.shared)
         self.dims = M.make_dims(cfg.T, cfg.d, cfg.F, cfg.E, cfg.k,
                                 M.MOE_ROUTE_HASH if cfg.route == "hash" else M.MOE_ROUTE_SOFTMAX_TOPK,
-                                M.MOE_A_MXFP8 if cfg.act == "mxfp8" else M.MOE_A_BF16,
+                                {"mxfp8": M.MOE_A_MXFP8, "mxfp4": M.MOE_A_MXFP4}.get(cfg.act, M.MOE_A_BF16),
                                 M.MOE_W_Q2K if cfg.wfmt == "q2k" else M.MOE_W_MXFP4,
                                 cfg.Fs if self.shared is not None else 0)
         dev = torch.device("cuda:0")
