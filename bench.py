@@ -154,35 +154,54 @@ def algorithmic_ffn_bytes(cfg, n_experts_touched):
     return per * n_experts_touched + 3 * cfg.Fs * cfg.d * 2
 
 
-# DRAM traffic of one decode_ffn_kernel launch on batch 0 of the default
-# workload (decode T=8, 256 experts, 58 of them touched): dram__bytes_read.sum +
-# dram__bytes_write.sum from a one-pass ncu capture of that launch (826.33 +
-# 4.47 MB as ncu printed them; command and figures in
-# profiles/decode_ffn_kernel_traffic_decode_T8.md). The figure belongs to the
-# sources it was taken on: their SHA-256 is checked before it is reported.
-DECODE_TRAFFIC = {
-    "T": 8, "E": 256, "dram_bytes": 830_800_000,
-    "sources": ["routed_expert_ffn_05_b200/csrc/decode.cu", "routed_expert_ffn_05_b200/csrc/common.cuh",
-                "routed_expert_ffn_05_b200/csrc/kernels.h", "routed_expert_ffn_05_b200/csrc/ptx.cuh",
-                "routed_expert_ffn_05_b200/csrc/tma.h", "routed_expert_ffn_05_b200/csrc/tma.cu",
-                "routed_expert_ffn_05_b200/csrc/layout.h", "include/moe.h"],
-    "sources_sha256": "d8dad1616d9e0f2d1e26667a34b0d83a67afe39cecd892a08e98ddf7852e90d4",
-}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) from one-pass ncu
+# captures of full-size launches, one record per workload. Each figure belongs
+# to the sources it was taken on: their SHA-256 is checked before it is
+# reported, and the field is null once any of them has changed.
+#  - decode T=8: one decode_ffn_kernel launch on batch 0 (58 experts touched);
+#    command and figures in profiles/decode_ffn_kernel_traffic_decode_T8.md.
+#  - prefill T=4096 (w4a8): the gate/up and the down tc_ffn_kernel launches of
+#    one layer call (batch 2), summed: 1,684.8 + 1,054.5 MB; command and figures
+#    in profiles/tc_ffn_kernel_traffic_prefill_T4096.md.
+_DECODE_SOURCES = ["routed_expert_ffn_05_b200/csrc/decode.cu", "routed_expert_ffn_05_b200/csrc/common.cuh",
+                   "routed_expert_ffn_05_b200/csrc/kernels.h", "routed_expert_ffn_05_b200/csrc/ptx.cuh",
+                   "routed_expert_ffn_05_b200/csrc/tma.h", "routed_expert_ffn_05_b200/csrc/tma.cu",
+                   "routed_expert_ffn_05_b200/csrc/layout.h", "include/moe.h"]
+_PREFILL_SOURCES = ["routed_expert_ffn_05_b200/csrc/prefill.cu", "routed_expert_ffn_05_b200/csrc/tc.cuh",
+                    "routed_expert_ffn_05_b200/csrc/common.cuh", "routed_expert_ffn_05_b200/csrc/kernels.h",
+                    "routed_expert_ffn_05_b200/csrc/ptx.cuh", "routed_expert_ffn_05_b200/csrc/tma.h",
+                    "routed_expert_ffn_05_b200/csrc/tma.cu", "routed_expert_ffn_05_b200/csrc/layout.h",
+                    "include/moe.h"]
+TRAFFIC = [
+    {"config": "decode", "T": 8, "E": 256, "act": "bf16", "dram_bytes": 830_800_000,
+     "kernels": "decode_ffn_kernel<MXFP4>", "sources": _DECODE_SOURCES,
+     "sources_sha256": "d8dad1616d9e0f2d1e26667a34b0d83a67afe39cecd892a08e98ddf7852e90d4"},
+    {"config": "prefill", "T": 4096, "E": 256, "act": "mxfp8", "dram_bytes": 2_739_271_424,
+     "kernels": "tc_ffn_kernel gate/up + down", "sources": _PREFILL_SOURCES,
+     "sources_sha256": "1bc0465f6a1b8c910b2aa5dac407c8870298f965d9ecde875e2ecb7b524d7a26"},
+]
 
 
-def decode_traffic(cfg, T):
-    """The captured per-launch DRAM bytes when this run is that workload on the
-    captured sources, else None."""
-    rec = DECODE_TRAFFIC
-    if not (cfg.wfmt == "mxfp4" and cfg.act == "bf16" and cfg.route == "softmax" and T == rec["T"]
-            and cfg.E == rec["E"] and cfg.d == 4096 and cfg.F == 2048 and cfg.Fs == 2048):
-        return None
+def sources_sha256(files):
     import hashlib
     h = hashlib.sha256()
-    for f in rec["sources"]:
+    for f in files:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
-    return rec["dram_bytes"] if h.hexdigest() == rec["sources_sha256"] else None
+    return h.hexdigest()
+
+
+def captured_traffic(cfg, T):
+    """The captured per-launch DRAM bytes (and the kernels they cover) when this
+    run is a captured workload on the captured sources, else (None, None)."""
+    for rec in TRAFFIC:
+        base = synth.CONFIGS[rec["config"]]
+        if (cfg.wfmt == base.wfmt and cfg.act == rec["act"] and cfg.route == base.route and T == rec["T"]
+                and cfg.E == rec["E"] and cfg.d == base.d and cfg.F == base.F and cfg.Fs == base.Fs
+                and cfg.zipf_s == base.zipf_s):
+            if sources_sha256(rec["sources"]) == rec["sources_sha256"]:
+                return rec["dram_bytes"], rec["kernels"]
+    return None, None
 
 
 def hbm_fraction(M, torch, layer, cfg, T, r, hbm, rank):
@@ -509,7 +528,8 @@ def main():
                 "peak_source": f"{src} bf16" + (f" x {ratio:g} ({'FP8' if ratio == 2 else 'FP4'} nominal ratio)"
                                                  if ratio != 1 else ""),
                 "frac_of_fp4_peak": achieved / (4.0 * bf16),
-                "traffic": None, "algorithmic_flops": fl, "ffn_ms": ffn_ms}
+                "traffic": captured_traffic(cfg, T)[0], "traffic_kernels": captured_traffic(cfg, T)[1],
+                "algorithmic_flops": fl, "ffn_ms": ffn_ms}
     else:
         xb = torch.from_numpy(synth.make_x(cfg, 0, 1000 * (0 if ep else rank)).astype(np.int16)).cuda()
         idx = touched_experts(M, torch, layer, xb, None, T)
@@ -521,7 +541,7 @@ def main():
         achieved = alg / (ffn_ms / 1000.0) / 1e9
         roof = {"kernel": "expert FFN: routed + shared", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_source": src, "traffic": decode_traffic(cfg, T),
+                "peak_source": src, "traffic": captured_traffic(cfg, T)[0],
                 "algorithmic_bytes": alg, "experts_touched": U, "ffn_ms": ffn_ms}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -581,6 +601,13 @@ def main():
         tps, threads, el, desc = oracle_sample(cfg, T, n_cpu_tokens, 10.0)
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": desc, "seconds": el}
+        # the same oracle on one thread (a single-threaded C loop over the tokens)
+        import oracle
+        oracle.set_num_threads(1)
+        tps1, threads1, el1, desc1 = oracle_sample(cfg, T, 1, 5.0)
+        oracle.set_num_threads(threads)
+        line["cpu_baseline"]["single_thread"] = {"value": tps1, "unit": UNIT, "cores": threads1,
+                                                 "sample": desc1, "seconds": el1}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -84,6 +84,7 @@ def lib():
             "ora_combine": (None, [vp, vp, vp, vp, i32, i32, i32, vp]),
             "ora_layer_tokens": (i32, [vp, vp, vp, vp, i32, vp, vp, vp]),
             "ora_num_threads": (i32, []),
+            "ora_set_num_threads": (i32, [i32]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -101,6 +102,12 @@ def _p(a):
 
 def num_threads() -> int:
     return int(lib().ora_num_threads())
+
+
+def set_num_threads(n: int) -> int:
+    """OpenMP threads for later calls (threading only; results do not depend
+    on it). Returns the count in effect."""
+    return int(lib().ora_set_num_threads(int(n)))
 
 
 # ---- formats ---------------------------------------------------------------

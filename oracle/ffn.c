@@ -41,6 +41,17 @@ int ora_num_threads(void) {
 #endif
 }
 
+/* Threads of later parallel regions (n >= 1); returns the count then in effect.
+ * Threading only: every result is the same at any count. */
+int ora_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+    return ora_num_threads();
+}
+
 static double silu(double g) { return g / (1.0 + exp(-g)); }
 
 /* sum_i a[i] * W[n][i] for an MXFP4 row: codes [K/2], scales [K/32]. */

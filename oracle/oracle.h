@@ -107,6 +107,7 @@ int ora_layer_tokens(const ora_layer *L, const uint16_t *x, const int32_t *token
                      const int32_t *tokens, int n_tokens, int32_t *idx, float *w, float *y);
 
 int ora_num_threads(void);
+int ora_set_num_threads(int n);   /* threading only; returns the count in effect */
 
 #ifdef __cplusplus
 }
