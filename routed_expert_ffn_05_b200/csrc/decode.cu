@@ -75,8 +75,11 @@ constexpr int kD = 4096, kF = 2048;       // the dims this tiling is written for
 constexpr int kGuTiles = kF / 16;         // gate/up tiles per routed expert
 // A routed down unit: 64 W2 rows over all K (two stages of 32 rows) for
 // MXFP4, 32 rows (one stage) for Q2_K; its partial tiles are 16 rows each.
+// (A 64-row Q2_K unit in one stage, with three stages to make room for its
+// partial tiles, measured 1% faster at T = 8 and 5% slower at T = 1.)
 template <int WF> constexpr int dn_rows() { return WF == MOE_W_Q2K ? 32 : 64; }
-template <int WF> constexpr int dn_stages() { return dn_rows<WF>() / 32; }
+template <int WF> constexpr int dn_parts() { return dn_rows<WF>() / 32; }
+template <int WF> constexpr int dn_stages() { return dn_parts<WF>(); }
 template <int WF> constexpr int dn_tiles() { return kD / dn_rows<WF>(); }
 template <int WF> constexpr int red_w() { return dn_rows<WF>() / 16 * kRedM; }  // floats per warp
 constexpr int kDshTiles = kD / 16;        // shared-expert down tiles
@@ -301,57 +304,51 @@ __device__ __forceinline__ float row_scale(uint32_t hm) {  // 2^p with max |h| *
 }
 
 // ---- Q2_K ----
-// Quants are stored in lane order (see layout.h): the 32-bit word 4G + q of a
-// super-block holds lane q's quants of sub-blocks 4G .. 4G + 3 as 8 pairs,
-// pair k = 2 (sub-block % 4) + h with its two quants 16 bits apart. MMA k-slots
-// 2q, 2q+1 carry elements 4q, 4q+1 of a 16-element sub-block (h = 0) and
-// k-slots 2q+8, 2q+9 elements 4q+2, 4q+3 (h = 1). Pair k is masked out of the
-// word shifted by 6 (k / 3), at bit 2 (k % 3), so it carries 4^(k % 3) q; an
-// integer multiply by the sub-block scale sc gives sc q 4^(k % 3) <= 720 in
-// each 16-bit half, used directly as an f16 subnormal (value x 2^-24, exact).
-// The activation k-slots of pair k are pre-scaled by 4^-(k % 3).
-template <int K>
-__device__ __forceinline__ uint32_t q2_pair(uint32_t w, uint32_t sc) {
-    return ((w >> (6 * (K / 3))) & (0x00030003u << (2 * (K % 3)))) * sc;
-}
-__host__ __device__ constexpr float q2_pre(int k) { return k % 3 == 0 ? 1.0f : (k % 3 == 1 ? 0.25f : 0.0625f); }
+// The main term runs on integer MMAs (m16n8k32, u8 x s8 and u8 x u8 -> s32).
+// A is sc q (<= 45) per byte: the lane's quant word (lane order, layout.h)
+// shifted and masked to four bytes, times the sub-block scale sc in one 32-bit
+// multiply (no carry crosses a byte). B is the activation as an integer
+// X = round(x 2^-p), |X| < 2^15 (p puts the row's largest |x| in [2^14, 2^15),
+// so every element within 2^7 of it is exact), split into a signed high byte
+// and an unsigned low byte, X = 256 hi + lo. The super-block's sum_k sc q X is
+// 256 c_hi + c_lo, exact in 32 bits (< 2^29); d scales it once in fp32.
 
 // One super-block (16 sub-blocks of 16), or half of one (HALF 0: sub-blocks
-// 0..7, HALF 1: 8..15; HALF -1: all), of 16 rows r0 + g, r0 + g + 8 of a Q2_K
-// box (quants: `rows` rows, 128-byte chunks; sc|m: same rows, chunked; dd:
-// row-major, `ddrow` bytes per row) against B (this part's sub-blocks) and bm
-// (sub-block sums as f16 hi + lo parts: bm[0..1] hi, bm[2..3] lo).
-// acc += d (sum_j sc_j q . x) - dmin (sum_j m_j xsum_j) over the part.
+// 0..7, HALF 1: 8..15; HALF -1: all), of 16 rows r0 + sigma(g), r0 + sigma(g)
+// + 8 of a Q2_K box (quants: `rows` rows, 128-byte chunks; sc|m: same rows,
+// chunked; dd: `ddrow` bytes per row, 64-byte swizzled for a whole super-block
+// (gate/up boxes), row-major for a half (down boxes)) against B (the part's K
+// steps of 32: high bytes in B[i][0..1], low bytes in B[i][2..3]) and bm
+// (sub-block sums as f16 hi + lo parts: bm[0..1] hi, bm[2..3] lo). MMA row g
+// reads shared row sigma(g): a quarter warp's 16-byte quant loads then fall on
+// 8 different bank groups; the partial tile puts it back at row sigma(g).
+// acc += d (sum_j sc_j q . X) - dmin (sum_j m_j Xsum_j) over the part.
 template <int HALF>
 __device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, const uint8_t *scm,
                                                const uint8_t *dd, int rows, int ddrow, int r0, int sb, int g,
                                                int q, const uint32_t (*B)[4], const uint32_t bm[4]) {
-    constexpr int G0 = HALF == 1 ? 2 : 0, NG = HALF < 0 ? 4 : 2;
-    const int rg = r0 + g, rh = r0 + g + 8;
+    constexpr int S0 = HALF == 1 ? 4 : 0, NS = HALF < 0 ? 8 : 4;
+    const int rg = r0 + sigma(g), rh = rg + 8;
     const uint4 ml = lds128(scm + swz_off((sb * 16) / 128, rows, rg, sb % 8));
     const uint4 mh = lds128(scm + swz_off((sb * 16) / 128, rows, rh, sb % 8));
+    const uint4 wl = lds128(qs + swz_off((sb * 64) / 128, rows, rg, 4 * (sb & 1) + q));
+    const uint4 wh = lds128(qs + swz_off((sb * 64) / 128, rows, rh, 4 * (sb & 1) + q));
     const uint32_t sl[4] = {ml.x, ml.y, ml.z, ml.w}, sh[4] = {mh.x, mh.y, mh.z, mh.w};
-    float tm[4];
+    const uint32_t ql[4] = {wl.x, wl.y, wl.z, wl.w}, qh[4] = {wh.x, wh.y, wh.z, wh.w};
+    int chi[4] = {0, 0, 0, 0}, clo[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int Gi = 0; Gi < NG; ++Gi) {
-        const int G = G0 + Gi;
-        const int c = (sb * 64) / 128, u = 4 * (sb & 1) + G;
-        const uint32_t wl = lds32(qs + swz_off(c, rows, rg, u) + 4 * q);
-        const uint32_t wh = lds32(qs + swz_off(c, rows, rh, u) + 4 * q);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const uint32_t cl = (sl[G] >> (8 * jj)) & 15u, ch = (sh[G] >> (8 * jj)) & 15u;
-            uint32_t a0, a1, a2, a3;
-            switch (jj) {  // pair indices are compile-time constants
-                case 0: a0 = q2_pair<0>(wl, cl); a1 = q2_pair<0>(wh, ch); a2 = q2_pair<1>(wl, cl); a3 = q2_pair<1>(wh, ch); break;
-                case 1: a0 = q2_pair<2>(wl, cl); a1 = q2_pair<2>(wh, ch); a2 = q2_pair<3>(wl, cl); a3 = q2_pair<3>(wh, ch); break;
-                case 2: a0 = q2_pair<4>(wl, cl); a1 = q2_pair<4>(wh, ch); a2 = q2_pair<5>(wl, cl); a3 = q2_pair<5>(wh, ch); break;
-                default: a0 = q2_pair<6>(wl, cl); a1 = q2_pair<6>(wh, ch); a2 = q2_pair<7>(wl, cl); a3 = q2_pair<7>(wh, ch);
-            }
-            const int jl = 4 * Gi + jj;  // sub-block within this part
-            if (jl == 0) mma_f16_16816_z(tm, a0, a1, a2, a3, B[0][0], B[0][1]);
-            else mma_f16_16816(tm, a0, a1, a2, a3, B[jl >> 1][2 * (jl & 1)], B[jl >> 1][2 * (jl & 1) + 1]);
-        }
+    for (int i = 0; i < NS; ++i) {
+        const int st = S0 + i;                   // K 32 st .. + 31: sub-blocks 2 st, 2 st + 1
+        const int w = st >> 1, sft = 4 * (st & 1), sb8 = 16 * (st & 1);
+        // their scales: low nibbles of bytes 2 (st % 2), 2 (st % 2) + 1 of sc|m word st / 2
+        const uint32_t s0l = (sl[w] >> sb8) & 15u, s1l = (sl[w] >> (sb8 + 8)) & 15u;
+        const uint32_t s0h = (sh[w] >> sb8) & 15u, s1h = (sh[w] >> (sb8 + 8)) & 15u;
+        const uint32_t a0 = ((ql[w] >> sft) & 0x03030303u) * s0l;
+        const uint32_t a1 = ((qh[w] >> sft) & 0x03030303u) * s0h;
+        const uint32_t a2 = ((ql[w] >> (sft + 2)) & 0x03030303u) * s1l;
+        const uint32_t a3 = ((qh[w] >> (sft + 2)) & 0x03030303u) * s1h;
+        mma_u8s8_16832(chi, a0, a1, a2, a3, B[i][0], B[i][1]);
+        mma_u8u8_16832(clo, a0, a1, a2, a3, B[i][2], B[i][3]);
     }
     // minimum term: A = m of sub-blocks 2q, 2q+1 (k-slots 2q, 2q+1) and 2q+8, 2q+9;
     // a half keeps only its own sub-blocks
@@ -366,50 +363,57 @@ __device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, 
     float tn[4];
     mma_f16_16816_z(tn, ma0, ma1, ma2, ma3, bm[0], bm[1]);
     mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[2], bm[3]);
-    const uint32_t dl = lds32(dd + rg * ddrow + 4 * sb), dh = lds32(dd + rh * ddrow + 4 * sb);
-    // 2^24 undoes the subnormal encoding; 2^5 the sub-block-sum pre-scale
-    const float d0 = __half2float(__ushort_as_half((uint16_t)(dl & 0xFFFF))) * 16777216.0f;
+    const uint32_t dl = lds32(dd + (HALF < 0 ? scale_off(rg, sb) : rg * ddrow + 4 * sb));
+    const uint32_t dh = lds32(dd + (HALF < 0 ? scale_off(rh, sb) : rh * ddrow + 4 * sb));
+    // dmin: 2^24 undoes the subnormal encoding of m, 2^5 the sub-block-sum pre-scale
+    const float d0 = __half2float(__ushort_as_half((uint16_t)(dl & 0xFFFF)));
     const float m0 = __half2float(__ushort_as_half((uint16_t)(dl >> 16))) * 536870912.0f;
-    const float d1 = __half2float(__ushort_as_half((uint16_t)(dh & 0xFFFF))) * 16777216.0f;
+    const float d1 = __half2float(__ushort_as_half((uint16_t)(dh & 0xFFFF)));
     const float m1 = __half2float(__ushort_as_half((uint16_t)(dh >> 16))) * 536870912.0f;
-    acc[0] = fmaf(-m0, tn[0], fmaf(d0, tm[0], acc[0]));
-    acc[1] = fmaf(-m0, tn[1], fmaf(d0, tm[1], acc[1]));
-    acc[2] = fmaf(-m1, tn[2], fmaf(d1, tm[2], acc[2]));
-    acc[3] = fmaf(-m1, tn[3], fmaf(d1, tm[3], acc[3]));
+    acc[0] = fmaf(-m0, tn[0], fmaf(d0, __int2float_rn(256 * chi[0] + clo[0]), acc[0]));
+    acc[1] = fmaf(-m0, tn[1], fmaf(d0, __int2float_rn(256 * chi[1] + clo[1]), acc[1]));
+    acc[2] = fmaf(-m1, tn[2], fmaf(d1, __int2float_rn(256 * chi[2] + clo[2]), acc[2]));
+    acc[3] = fmaf(-m1, tn[3], fmaf(d1, __int2float_rn(256 * chi[3] + clo[3]), acc[3]));
 }
 
 // B fragments of one super-block, or half of one (HALF as above), of an
 // activation row (bf16 at `row` = the super-block's first element, scaled by
-// `inv`): k-slot pre-scale 4^-(k % 3), the elements of lane q as described
-// above; bm gets the sums (scaled by 2^-5) of sub-blocks 2q, 2q+1, 2q+8, 2q+9
-// that lie in the part (zero otherwise), each split into an f16 part and the
-// f16 of its remainder (together ~22 bits: the minimum term nearly cancels
-// the main term, so its sums need more than f16).
+// `inv` into integers X as described above): step i's k-slots 4q .. 4q + 3 of
+// sub-blocks 2 (S0 + i) and 2 (S0 + i) + 1, high bytes in B[i][0..1], low bytes
+// in B[i][2..3]; bm gets the sums (scaled by 2^-5) of X over sub-blocks 2q,
+// 2q+1, 2q+8, 2q+9 that lie in the part (zero otherwise), each split into an
+// f16 part and the f16 of its remainder (exact: the sums are integers below
+// 2^19, and the minimum term nearly cancels the main term, so it needs them
+// whole).
 template <int HALF, bool CG>
 __device__ __forceinline__ void q2k_load_b(const uint16_t *row, float inv, int q, uint32_t (*B)[4], uint32_t bm[4]) {
-    constexpr int J0 = HALF == 1 ? 8 : 0, NJ = HALF < 0 ? 16 : 8;
-    float keep[4] = {0.f, 0.f, 0.f, 0.f};
+    constexpr int S0 = HALF == 1 ? 4 : 0, NS = HALF < 0 ? 8 : 4;
+    int keep[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int ji = 0; ji < NJ; ++ji) {
-        const int j = J0 + ji;
-        const uint16_t *src = row + 16 * j + 4 * q;
-        const uint2 v = CG ? __ldcg(reinterpret_cast<const uint2 *>(src)) : __ldg(reinterpret_cast<const uint2 *>(src));
-        const float x0 = __uint_as_float(v.x << 16), x1 = __uint_as_float(v.x & 0xFFFF0000u);
-        const float x2 = __uint_as_float(v.y << 16), x3 = __uint_as_float(v.y & 0xFFFF0000u);
-        const float c0 = inv * q2_pre(2 * (j & 3)), c1 = inv * q2_pre(2 * (j & 3) + 1);
-        B[ji >> 1][2 * (ji & 1)] = f32x2_to_f16x2(x0 * c0, x1 * c0);
-        B[ji >> 1][2 * (ji & 1) + 1] = f32x2_to_f16x2(x2 * c1, x3 * c1);
-        float ps = (x0 + x1) + (x2 + x3);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-        if (j < 8 && (j >> 1) == q) keep[j & 1] = ps;
-        if (j >= 8 && ((j - 8) >> 1) == q) keep[2 + (j & 1)] = ps;
+    for (int i = 0; i < NS; ++i) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int j = 2 * (S0 + i) + h;  // sub-block
+            const uint16_t *src = row + 16 * j + 4 * q;
+            const uint2 v = CG ? __ldcg(reinterpret_cast<const uint2 *>(src)) : __ldg(reinterpret_cast<const uint2 *>(src));
+            const int X0 = __float2int_rn(__uint_as_float(v.x << 16) * inv);
+            const int X1 = __float2int_rn(__uint_as_float(v.x & 0xFFFF0000u) * inv);
+            const int X2 = __float2int_rn(__uint_as_float(v.y << 16) * inv);
+            const int X3 = __float2int_rn(__uint_as_float(v.y & 0xFFFF0000u) * inv);
+            // byte 1 (high) and byte 0 (low) of each 16-bit two's-complement X
+            B[i][h] = __byte_perm(__byte_perm(X0, X1, 0x0051), __byte_perm(X2, X3, 0x0051), 0x5410);
+            B[i][2 + h] = __byte_perm(__byte_perm(X0, X1, 0x0040), __byte_perm(X2, X3, 0x0040), 0x5410);
+            int ps = (X0 + X1) + (X2 + X3);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+            if (j < 8 && (j >> 1) == q) keep[j & 1] = ps;
+            if (j >= 8 && ((j - 8) >> 1) == q) keep[2 + (j & 1)] = ps;
+        }
     }
-    const float xs = inv * 0.03125f;
     float hi[4], lo[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float v = keep[i] * xs;
+        const float v = (float)keep[i] * 0.03125f;  // exact: |keep| < 2^19
         hi[i] = __half2float(__float2half_rn(v));
         lo[i] = v - hi[i];
     }
@@ -711,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     dsc = lane < cnt ? row_scale(__ldcg(&a.hmax[rbase + lane])) : 1.f;
                 }
 #pragma unroll
-                for (int p = 0; p < dn_stages<WF>(); ++p)
+                for (int p = 0; p < dn_parts<WF>(); ++p)
                     for (int i = 0; i < cnt; ++i) {
                         const float sc = __shfl_sync(0xffffffffu, dsc, i);
                         a.out_rows[(int64_t)(rbase + i) * kD + dn_rows<WF>() * un.tile + 32 * p + lane] =
@@ -944,7 +948,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         const int rb = ru & 1;
         if (Q2 || un.kind != kDrt) {
             if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1, &s.abort)) { fail(a, s); return; }
-            const int rg = (un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;  // bf16 tiles read rows sigma(g)
+            // bf16 and Q2_K tiles read rows sigma(g)
+            const int rg = (Q2 || un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;
             put_partial(s.red[rb][warp], rg, q, acc[0]);
             if (un.kind != kDsh) put_partial(s.red[rb][warp] + kRedM, rg, q, acc[1]);
         }
@@ -1246,8 +1251,8 @@ cudaError_t launch_decode_ffn(const moe_dims &d, const moe_weights &w, const uin
              make_chunked_map(&a.m1s, p1 + L1.scm, r13, kD / 16, 16, 2) &&
              make_chunked_map(&a.m3s, p3 + L1.scm, r13, kD / 16, 16, 2) &&
              make_chunked_map(&a.m2s, p2 + L2.scm, r2, kF / 16, 32, 1) &&
-             make_plain_map(&a.m1d, p1 + L1.dd, r13, kD / 64, kD / 64, 16) &&
-             make_plain_map(&a.m3d, p3 + L1.dd, r13, kD / 64, kD / 64, 16) &&
+             make_plain_map(&a.m1d, p1 + L1.dd, r13, kD / 64, kD / 64, 16, true) &&
+             make_plain_map(&a.m3d, p3 + L1.dd, r13, kD / 64, kD / 64, 16, true) &&
              make_plain_map(&a.m2d, p2 + L2.dd, r2, kF / 64, kF / 64, 32);
     } else {
         const Mxfp4Layout L1 = mxfp4_layout(d, MOE_MAT_W1), L2 = mxfp4_layout(d, MOE_MAT_W2);

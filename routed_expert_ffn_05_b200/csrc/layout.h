@@ -48,17 +48,18 @@ MOE_HD static inline int64_t mxfp4_tile_index(int64_t e, int64_t n, int64_t kb, 
 // Packed Q2_K matrix: quants [E][N][K/256][64], sc|m<<4 bytes [E][N][K/256][16],
 // (d, dmin) fp16 pairs [E][N][K/256].
 //
-// The 64 quant bytes of a super-block are 16 32-bit words in "lane order":
-// quant e (0..255; sub-block j = e / 16) sits in word 4 (e / 64) + (e % 16) / 4
-// at bit 2 (2 (j % 4) + (e % 4) / 2) + 16 (e % 2). Word 4G + q holds the 16
-// quants that lane q of an MMA quad needs from sub-blocks 4G .. 4G + 3
-// (elements 4q .. 4q + 3 of each), as 8 pairs with the pair's two quants 16
-// bits apart: one mask gives both halves of a packed 16-bit pair.
+// The 64 quant bytes of a super-block are 16 32-bit words in "lane order" for
+// the integer MMA m16n8k32 (K 32 = two sub-blocks per MMA): quant e (0..255;
+// sub-block c = e / 16) sits in word 4 ((e % 16) / 4) + c / 4 at bit
+// 8 (e % 4) + 2 (c % 4). Lane q of an MMA quad reads words 4q .. 4q + 3 (16
+// bytes), which hold elements 4q .. 4q + 3 of every sub-block; word 4q + c / 4
+// shifted right by 2 (c % 4) and masked with 0x03030303 gives those four
+// quants of sub-block c as four bytes, the A-fragment order of the MMA.
 struct Q2kLayout {
     int64_t N, K, E, qs, scm, dd, total;
 };
-MOE_HD static inline int q2k_word(int e) { return 4 * (e / 64) + (e % 16) / 4; }
-MOE_HD static inline int q2k_bit(int e) { return 2 * (2 * ((e / 16) % 4) + (e % 4) / 2) + 16 * (e % 2); }
+MOE_HD static inline int q2k_word(int e) { return 4 * ((e % 16) / 4) + (e / 16) / 4; }
+MOE_HD static inline int q2k_bit(int e) { return 8 * (e % 4) + 2 * ((e / 16) % 4); }
 
 static inline Q2kLayout q2k_layout(const moe_dims &d, int which) {
     Q2kLayout L;

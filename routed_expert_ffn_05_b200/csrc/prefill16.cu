@@ -13,7 +13,10 @@
 //  - A = 128 weight rows, decoded into TENSOR memory by four decoder warps
 //    (thread = weight row = TMEM lane: 64 codes and two scales per stage become
 //    32 bf16 pairs, one tcgen05.st of 32 columns), so the decoded tile never
-//    passes through shared memory;
+//    passes through shared memory; the packed codes arrive by TMA (32 bytes
+//    per row and stage) in the same shared-memory stage as the token rows,
+//    with the tile's E8M0 scale atom (128 rows x K 128, the layout the
+//    block-scaled path reads) beside them;
 //  - B = a tile of 128 of the expert's token rows (bf16, K-major, 128-byte
 //    swizzled TMA boxes of K = 64); gate/up: the gathered x rows, down: h;
 //  - gate/up runs two MMAs per K step into two accumulators (g from W1 rows,
@@ -21,8 +24,10 @@
 //  - the epilogue thread is a weight row (TMEM lane), its columns tokens:
 //    h = bf16(silu(g) u) goes to h [S][d_ff] (K-major for the down GEMM), the
 //    down rows to out_rows [S][d_model] in fp32.
-// One persistent CTA per SM: a TMA warp, an MMA warp, four decoder warps and
-// eight epilogue warps; a 4-stage ring; every wait is bounded.
+// One persistent CTA per SM: a TMA warp, an MMA warp, twelve decoder warps
+// (three per TMEM lane quarter, taking the stages in turn) and four epilogue
+// warps; an 8-stage shared-memory ring (token rows + codes) ahead of a 4-stage
+// tensor-memory ring (decoded A); every wait is bounded.
 #include <string.h>
 
 #include <atomic>
@@ -37,8 +42,10 @@
 namespace moe {
 namespace {
 
-constexpr int k16Stages = 4;
-constexpr int k16Threads = 448;   // warp 0 TMA, 1 MMA, 2..5 decoders, 6..13 epilogue
+constexpr int k16Sm = 8;          // shared-memory stages: token rows and weight codes
+constexpr int k16Ta = 4;          // tensor-memory stages: decoded weights
+constexpr int k16Dec = 3;         // decoder warps per TMEM lane quarter (they take turns by stage)
+constexpr int k16Threads = 576;   // warp 0 TMA, 1 MMA, 2..13 decoders, 14..17 epilogue
 constexpr int k16Tile = 128;      // weight rows (M) and tokens (N) per tile
 constexpr int k16Kst = 64;        // K per stage (one 128-byte row of bf16)
 constexpr int k16MaxE = 1024;
@@ -48,8 +55,9 @@ enum { kGU16 = 0, kDN16 = 1 };
 
 struct T16Args {
     CUtensorMap act;              // token rows bf16 [S][K], 64 x 128 boxes, 128-byte swizzled
-    const uint8_t *wc[2];         // packed E2M1 codes [E * Nw][K / 2]: gate/up W1, W3; down W2
-    const uint8_t *wsc[2];        // row-major E8M0 scales [E * Nw][K / 32]
+    CUtensorMap wcm[2];           // packed E2M1 codes [E * Nw][K / 2], 32-byte x 128-row boxes, 32-byte
+                                  // swizzled: gate/up W1, W3; down W2
+    const uint8_t *wsf[2];        // E8M0 scale atoms [E][Nw / 128][K / 128][512] (layout.h)
     const int32_t *offsets, *ustart;
     int E, Nw, K;                 // weight rows per expert, input dim
     uint16_t *h;                  // gate/up: h bf16 [S][Nw]
@@ -58,8 +66,10 @@ struct T16Args {
 };
 
 struct T16Smem {
-    uint8_t b[k16Stages][k16Tile * 128];
-    uint64_t b_full[k16Stages], a_full[k16Stages], empty[k16Stages], acc_full, acc_empty, mma_done;
+    uint8_t b[k16Sm][k16Tile * 128];      // token rows: 128 rows x K 64 (bf16)
+    uint8_t wc[k16Sm][2][k16Tile * 32];   // weight codes: 128 rows x K 64 (E2M1) per matrix
+    uint8_t wsf[k16Sm][2][512];           // the scale atom holding the stage's K 64 per matrix
+    uint64_t full[k16Sm], sempty[k16Sm], a_full[k16Ta], aempty[k16Ta], acc_full, acc_empty, mma_done;
     uint32_t tmem_base;
     volatile int abort;
     int ustart[k16MaxE + 1];
@@ -106,6 +116,17 @@ __device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
     return r;
 }
 
+// (lo, hi) * (s, s) as one packed fp32 multiply, round to nearest even.
+__device__ __forceinline__ float2 mul_f32x2(float2 v, float sc) {
+    uint64_t p, q, r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(p) : "f"(v.x), "f"(v.y));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(q) : "f"(sc));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(p), "l"(q));
+    float2 o;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+    return o;
+}
+
 // 64 E2M1 codes (32 bytes, element 2i in the low nibble of byte i) of one
 // weight row and their two E8M0 scales -> 32 bf16 pairs, element order.
 __device__ __forceinline__ void decode64(const uint4 c[2], uint32_t sc2, uint32_t (&o)[32]) {
@@ -119,8 +140,8 @@ __device__ __forceinline__ void decode64(const uint4 c[2], uint32_t sc2, uint32_
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
             const __half2 h2 = *reinterpret_cast<const __half2 *>(&hh[b]);
-            const float2 f = __half22float2(h2);
-            o[4 * i + b] = f32x2_to_bf16x2(f.x * sc, f.y * sc);
+            const float2 f = mul_f32x2(__half22float2(h2), sc);
+            o[4 * i + b] = f32x2_to_bf16x2(f.x, f.y);
         }
     }
 }
@@ -137,13 +158,16 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
     const int ft = a.Nw / k16Tile, kt_n = a.K / k16Kst;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < k16Stages; ++i) {
-            mbar_init(&s.b_full[i], 1);
+        for (int i = 0; i < k16Sm; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.sempty[i], 1);
+        }
+        for (int i = 0; i < k16Ta; ++i) {
             mbar_init(&s.a_full[i], 4);  // one arrival per decoder warp
-            mbar_init(&s.empty[i], 1);
+            mbar_init(&s.aempty[i], 1);
         }
         mbar_init(&s.acc_full, 1);
-        mbar_init(&s.acc_empty, 8);
+        mbar_init(&s.acc_empty, 4);
         mbar_init(&s.mma_done, 1);
         s.abort = 0;
         fence_mbar_init();
@@ -160,21 +184,30 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
     const int n_work = ft * s.ustart[a.E];
 
     if (warp == 0) {
-        // ------------------------------ TMA: token rows ------------------------------
+        // ---------------------- TMA: token rows and weight codes ----------------------
         if (lane == 0) {
             prefetch_tensormap(&a.act);
+            prefetch_tensormap(&a.wcm[0]);
+            if (GU) prefetch_tensormap(&a.wcm[1]);
             int it = 0;
             for (int w = blockIdx.x; w < n_work && !s.abort; w += gridDim.x) {
                 const Work16 wk = work16_of(w, ft, s.ustart, a.E, a.offsets);
+                const int wrow = wk.e * a.Nw + wk.f * k16Tile;
                 for (int kt = 0; kt < kt_n; ++kt, ++it) {
-                    const int slot = it % k16Stages;
-                    if (!mbar_wait(&s.empty[slot], ((it / k16Stages) & 1) ^ 1, &s.abort)) { t16_fail(a, s); break; }
-                    mbar_arrive_expect_tx(&s.b_full[slot], k16Tile * 128);
-                    tma_load_2d(s.b[slot], &a.act, kt * 128, wk.row0, &s.b_full[slot]);
+                    const int slot = it % k16Sm;
+                    if (!mbar_wait(&s.sempty[slot], ((it / k16Sm) & 1) ^ 1, &s.abort)) { t16_fail(a, s); break; }
+                    mbar_arrive_expect_tx(&s.full[slot], k16Tile * 128 + kMats * (k16Tile * 32 + 512));
+                    tma_load_2d(s.b[slot], &a.act, kt * 128, wk.row0, &s.full[slot]);
+                    const int64_t atom = ((int64_t)wrow / k16Tile) * (a.K / 128) + (kt >> 1);
+#pragma unroll
+                    for (int m = 0; m < kMats; ++m) {
+                        tma_load_2d(s.wc[slot][m], &a.wcm[m], kt * 32, wrow, &s.full[slot]);
+                        bulk_g2s(s.wsf[slot][m], a.wsf[m] + atom * 512, 512, &s.full[slot]);
+                    }
                 }
             }
-            for (int g = it - k16Stages; g < it; ++g)  // copies in flight land before the CTA exits
-                if (g >= 0) mbar_wait(&s.b_full[g % k16Stages], (g / k16Stages) & 1);
+            for (int g = it - k16Sm; g < it; ++g)  // copies in flight land before the CTA exits
+                if (g >= 0) mbar_wait(&s.full[g % k16Sm], (g / k16Sm) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ------------------------------
@@ -186,22 +219,23 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < kt_n; ++kt, ++it) {
-                    const int slot = it % k16Stages;
-                    const uint32_t par = (it / k16Stages) & 1;
-                    if (!mbar_wait(&s.b_full[slot], par, &s.abort) || !mbar_wait(&s.a_full[slot], par, &s.abort)) {
+                    const int slot = it % k16Sm, ta = it % k16Ta;
+                    if (!mbar_wait(&s.full[slot], (it / k16Sm) & 1, &s.abort) ||
+                        !mbar_wait(&s.a_full[ta], (it / k16Ta) & 1, &s.abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint64_t db = sdesc_sw128(s.b[slot]);
-                    const uint32_t a0 = tmem + kAcc + kAStage * slot;
+                    const uint32_t a0 = tmem + kAcc + kAStage * ta;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {  // K = 16: 8 TMEM columns of A, 32 bytes of every B row
                         const uint32_t acc = (kt | ks) != 0;
                         tc_mma_bf16_ts(tmem, a0 + 8 * ks, db + 2 * ks, idesc, acc);
                         if (GU) tc_mma_bf16_ts(tmem + 128, a0 + 32 + 8 * ks, db + 2 * ks, idesc, acc);
                     }
-                    tc_commit(&s.empty[slot]);  // A columns and B stage free once these finish
+                    tc_commit(&s.sempty[slot]);  // the shared stage and
+                    tc_commit(&s.aempty[ta]);    // the A columns are free once these finish
                 }
                 if (!ok) { t16_fail(a, s); break; }
                 tc_commit(&s.acc_full);
@@ -209,63 +243,41 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
             tc_commit(&s.mma_done);
             mbar_wait(&s.mma_done, 0);
         }
-    } else if (warp < 6) {
+    } else if (warp < 2 + 4 * k16Dec) {
         // ------------------------------ decoders ------------------------------
         // thread = weight row r of the item's tile = TMEM lane r (this warp's
-        // lane quarter q); per stage 64 codes and 2 scales of each matrix
-        const int q = warp & 3, r = 32 * q + lane;
+        // lane quarter q); the warp decodes the stages with it % k16Dec == j:
+        // per stage the row's 32 code bytes of each matrix from the shared
+        // stage (32-byte swizzle: half c of row r at c ^ (r / 4 % 2)) and its
+        // four scale bytes of the atom (32-blocks 4 (kt / 2) .. + 3)
+        const int q = warp & 3, j = (warp - 2) >> 2, r = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        const int h0 = 16 * ((r >> 2) & 1), h1 = 16 - h0;  // byte offsets of the row's halves 0, 1
+        const int sfo = (r & 31) * 16 + (r >> 5) * 4;       // the row's scale word in an atom
         int it = 0;
         for (int w = blockIdx.x; w < n_work; w += gridDim.x) {
             if (__shfl_sync(0xffffffffu, s.abort, 0)) break;
-            const Work16 wk = work16_of(w, ft, s.ustart, a.E, a.offsets);
-            const int64_t grow = (int64_t)wk.e * a.Nw + (int64_t)wk.f * k16Tile + r;
-            const uint8_t *cp[kMats], *sp[kMats];
-#pragma unroll
-            for (int m = 0; m < kMats; ++m) {
-                cp[m] = a.wc[m] + grow * (a.K / 2);
-                sp[m] = a.wsc[m] + grow * (a.K / 32);
-            }
-            // the next stage's codes and scales are loaded before this one is decoded
-            uint4 c[kMats][2];
-            uint32_t sc[kMats];
-#pragma unroll
-            for (int m = 0; m < kMats; ++m) {
-                c[m][0] = __ldg(reinterpret_cast<const uint4 *>(cp[m]));
-                c[m][1] = __ldg(reinterpret_cast<const uint4 *>(cp[m]) + 1);
-                sc[m] = __ldg(reinterpret_cast<const uint16_t *>(sp[m]));
-            }
             bool ok = true;
             for (int kt = 0; kt < kt_n; ++kt, ++it) {
-                uint4 cn[kMats][2];
-                uint32_t sn[kMats];
-                const int kn = min(kt + 1, kt_n - 1);
-#pragma unroll
-                for (int m = 0; m < kMats; ++m) {
-                    cn[m][0] = __ldg(reinterpret_cast<const uint4 *>(cp[m] + 32 * kn));
-                    cn[m][1] = __ldg(reinterpret_cast<const uint4 *>(cp[m] + 32 * kn) + 1);
-                    sn[m] = __ldg(reinterpret_cast<const uint16_t *>(sp[m] + 2 * kn));
-                }
-                const int slot = it % k16Stages;
-                ok = mbar_wait(&s.empty[slot], ((it / k16Stages) & 1) ^ 1, &s.abort);
+                if (it % k16Dec != j) continue;
+                const int slot = it % k16Sm, ta = it % k16Ta;
+                ok = mbar_wait(&s.full[slot], (it / k16Sm) & 1, &s.abort) &&
+                     mbar_wait(&s.aempty[ta], ((it / k16Ta) & 1) ^ 1, &s.abort);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int m = 0; m < kMats; ++m) {
+                    const uint8_t *row = s.wc[slot][m] + 32 * r;
+                    const uint4 c[2] = {lds128(row + h0), lds128(row + h1)};
+                    const uint32_t sw = lds32(s.wsf[slot][m] + sfo) >> (16 * (kt & 1));  // bytes 2 (kt % 2), + 1
                     uint32_t o[32];
-                    decode64(c[m], sc[m], o);
-                    tmem_st32(lane_base + kAcc + kAStage * slot + 32 * m, o);
+                    decode64(c, sw, o);
+                    tmem_st32(lane_base + kAcc + kAStage * ta + 32 * m, o);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s.a_full[slot]);
-#pragma unroll
-                for (int m = 0; m < kMats; ++m) {
-                    c[m][0] = cn[m][0];
-                    c[m][1] = cn[m][1];
-                    sc[m] = sn[m];
-                }
+                if (lane == 0) mbar_arrive(&s.a_full[ta]);
             }
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) t16_fail(a, s);
@@ -275,8 +287,8 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
     } else {
         // ------------------------------ epilogue ------------------------------
         // TMEM lane = weight row (this warp: quarter q), columns = the tile's
-        // tokens; warp half hf takes tokens 64 hf .. 64 hf + 63.
-        const int q = warp & 3, hf = (warp - 6) >> 2, r = 32 * q + lane;
+        // tokens, in four chunks of 32.
+        const int q = warp & 3, r = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         int lw = 0;
         for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++lw) {
@@ -289,9 +301,9 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
             }
             tc_fence_after();
             const int col = wk.f * k16Tile + r;  // this thread's output feature (gate/up: row of h)
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int t0 = 64 * hf + 32 * cc;  // first token of this chunk
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                const int t0 = 32 * cc;            // first token of this chunk
                 if (t0 >= wk.nvalid) break;      // warp-uniform
                 uint32_t g[32], u[32];
                 tmem_ld32(lane_base + t0, g);
@@ -386,13 +398,17 @@ cudaError_t launch_tc16_ffn(const moe_dims &d, const moe_weights &w, const uint1
     T16Args g, dn;
     memset(&g, 0, sizeof g);
     memset(&dn, 0, sizeof dn);
+    const uint64_t r13 = (uint64_t)d.E * d.d_ff, r2 = (uint64_t)d.E * d.d_model;
     if (!make_tile_map_u8(&g.act, gx, S, (uint64_t)d.d_model * 2, k16Tile) ||
-        !make_tile_map_u8(&dn.act, h, S, (uint64_t)d.d_ff * 2, k16Tile))
+        !make_tile_map_u8(&dn.act, h, S, (uint64_t)d.d_ff * 2, k16Tile) ||
+        !make_rows32_map(&g.wcm[0], p1 + L1.codes, r13, (uint64_t)d.d_model / 2, k16Tile) ||
+        !make_rows32_map(&g.wcm[1], p3 + L1.codes, r13, (uint64_t)d.d_model / 2, k16Tile) ||
+        !make_rows32_map(&dn.wcm[0], p2 + L2.codes, r2, (uint64_t)d.d_ff / 2, k16Tile))
         return cudaErrorInvalidValue;
-    g.wc[0] = p1 + L1.codes; g.wc[1] = p3 + L1.codes; g.wsc[0] = p1 + L1.srow; g.wsc[1] = p3 + L1.srow;
+    g.wsf[0] = p1 + L1.stile; g.wsf[1] = p3 + L1.stile;
     g.offsets = offsets; g.ustart = ustart; g.E = d.E; g.Nw = d.d_ff; g.K = d.d_model; g.h = h;
     g.err = device_error_word();
-    dn.wc[0] = p2 + L2.codes; dn.wsc[0] = p2 + L2.srow;
+    dn.wsf[0] = p2 + L2.stile;
     dn.offsets = offsets; dn.ustart = ustart; dn.E = d.E; dn.Nw = d.d_model; dn.K = d.d_ff; dn.out = out_rows;
     dn.err = g.err;
     if ((e = launch_tc_plan(d, offsets, perm, ustart, row_of, s)) != cudaSuccess) return e;

@@ -25,6 +25,12 @@ bool make_chunked_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_
 bool make_plain_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_bytes,
                     uint32_t box_rows, bool swizzle64 = false);
 
+// A row-major byte matrix [rows][row_bytes] as 2D, boxes of 32 bytes x
+// box_rows rows, 32-byte swizzled: the 16-byte half c of box row r lands at
+// half c ^ ((r / 4) % 2), so the same half of 8 consecutive rows falls in 8
+// different groups of four banks (shared destination 256-byte aligned).
+bool make_rows32_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows);
+
 // Operand tiles for the tensor-core GEMMs: a row-major matrix [rows][K]
 // seen in boxes of 128 K-elements x box_rows rows, 128-byte swizzled (rows of
 // 128 bytes in shared memory, the K-major layout tcgen05.mma reads).
