@@ -315,65 +315,94 @@ __device__ __forceinline__ float row_scale(uint32_t hm) {  // 2^p with max |h| *
 
 // One super-block (16 sub-blocks of 16), or half of one (HALF 0: sub-blocks
 // 0..7, HALF 1: 8..15; HALF -1: all), of 16 rows r0 + sigma(g), r0 + sigma(g)
-// + 8 of a Q2_K box (quants: `rows` rows, 128-byte chunks; sc|m: same rows,
-// chunked; dd: `ddrow` bytes per row, 64-byte swizzled for a whole super-block
-// (gate/up boxes), row-major for a half (down boxes)) against B (the part's K
-// steps of 32: high bytes in B[i][0..1], low bytes in B[i][2..3]) and bm
-// (sub-block sums as f16 hi + lo parts: bm[0..1] hi, bm[2..3] lo). MMA row g
-// reads shared row sigma(g): a quarter warp's 16-byte quant loads then fall on
-// 8 different bank groups; the partial tile puts it back at row sigma(g).
-// acc += d (sum_j sc_j q . X) - dmin (sum_j m_j Xsum_j) over the part.
+// + 8 in each of two parts P[0], P[1] of Q2_K boxes (gate/up: the W1 and the W3
+// box; down: two 16-row tiles of one box), in lockstep, so four MMA chains are
+// in flight. A part's box: quants `rows` rows in 128-byte chunks; sc|m the same
+// rows, chunked; dd `ddrow` bytes per row, 64-byte swizzled for a whole
+// super-block (gate/up boxes), row-major for a half (down boxes). B holds the
+// part's K steps of 32 (high bytes in B[i][0..1], low bytes in B[i][2..3]); bm
+// the sub-block sums as f16 hi + lo parts (bm[0..1] hi, bm[2..3] lo). MMA row g
+// reads shared row sigma(g), so a quarter warp's 16-byte quant loads fall on 8
+// different bank groups; the partial tile puts it back at row sigma(g).
+// acc[p] += d (sum_j sc_j q . X) - dmin (sum_j m_j Xsum_j) over the part.
+struct Q2Part {
+    const uint8_t *qs, *scm, *dd;
+    int r0;
+};
 template <int HALF>
-__device__ __forceinline__ void q2k_superblock(float acc[4], const uint8_t *qs, const uint8_t *scm,
-                                               const uint8_t *dd, int rows, int ddrow, int r0, int sb, int g,
-                                               int q, const uint32_t (*B)[4], const uint32_t bm[4]) {
+__device__ __forceinline__ void q2k_superblock2(float (*acc)[4], const Q2Part (&P)[2], int rows, int ddrow, int sb,
+                                                int g, int q, const uint32_t (*B)[4], const uint32_t bm[4]) {
     constexpr int S0 = HALF == 1 ? 4 : 0, NS = HALF < 0 ? 8 : 4;
-    const int rg = r0 + sigma(g), rh = rg + 8;
-    const uint4 ml = lds128(scm + swz_off((sb * 16) / 128, rows, rg, sb % 8));
-    const uint4 mh = lds128(scm + swz_off((sb * 16) / 128, rows, rh, sb % 8));
-    const uint4 wl = lds128(qs + swz_off((sb * 64) / 128, rows, rg, 4 * (sb & 1) + q));
-    const uint4 wh = lds128(qs + swz_off((sb * 64) / 128, rows, rh, 4 * (sb & 1) + q));
-    const uint32_t sl[4] = {ml.x, ml.y, ml.z, ml.w}, sh[4] = {mh.x, mh.y, mh.z, mh.w};
-    const uint32_t ql[4] = {wl.x, wl.y, wl.z, wl.w}, qh[4] = {wh.x, wh.y, wh.z, wh.w};
-    int chi[4] = {0, 0, 0, 0}, clo[4] = {0, 0, 0, 0};
+    int rg[2], rh[2];
+    const uint8_t *qlp[2], *qhp[2], *slp[2], *shp[2];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-        const int st = S0 + i;                   // K 32 st .. + 31: sub-blocks 2 st, 2 st + 1
-        const int w = st >> 1, sft = 4 * (st & 1), sb8 = 16 * (st & 1);
-        // their scales: low nibbles of bytes 2 (st % 2), 2 (st % 2) + 1 of sc|m word st / 2
-        const uint32_t s0l = (sl[w] >> sb8) & 15u, s1l = (sl[w] >> (sb8 + 8)) & 15u;
-        const uint32_t s0h = (sh[w] >> sb8) & 15u, s1h = (sh[w] >> (sb8 + 8)) & 15u;
-        const uint32_t a0 = ((ql[w] >> sft) & 0x03030303u) * s0l;
-        const uint32_t a1 = ((qh[w] >> sft) & 0x03030303u) * s0h;
-        const uint32_t a2 = ((ql[w] >> (sft + 2)) & 0x03030303u) * s1l;
-        const uint32_t a3 = ((qh[w] >> (sft + 2)) & 0x03030303u) * s1h;
-        mma_u8s8_16832(chi, a0, a1, a2, a3, B[i][0], B[i][1]);
-        mma_u8u8_16832(clo, a0, a1, a2, a3, B[i][2], B[i][3]);
+    for (int p = 0; p < 2; ++p) {
+        rg[p] = P[p].r0 + sigma(g);
+        rh[p] = rg[p] + 8;
+        qlp[p] = P[p].qs + swz_off((sb * 64) / 128, rows, rg[p], 4 * (sb & 1) + q);
+        qhp[p] = P[p].qs + swz_off((sb * 64) / 128, rows, rh[p], 4 * (sb & 1) + q);
+        slp[p] = P[p].scm + swz_off((sb * 16) / 128, rows, rg[p], sb % 8);
+        shp[p] = P[p].scm + swz_off((sb * 16) / 128, rows, rh[p], sb % 8);
     }
-    // minimum term: A = m of sub-blocks 2q, 2q+1 (k-slots 2q, 2q+1) and 2q+8, 2q+9;
-    // a half keeps only its own sub-blocks
+    int chi[2][4], clo[2][4];
+#pragma unroll
+    for (int p = 0; p < 2; ++p)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) chi[p][i] = clo[p][i] = 0;
+#pragma unroll
+    for (int w = S0 / 2; w < (S0 + NS) / 2; ++w) {  // quant word w of the lane and sc|m word w: K steps 2w, 2w + 1
+        uint32_t ql[2], qh[2], sl[2], sh[2];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            ql[p] = lds32(qlp[p] + 4 * w);
+            qh[p] = lds32(qhp[p] + 4 * w);
+            sl[p] = lds32(slp[p] + 4 * w);
+            sh[p] = lds32(shp[p] + 4 * w);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int st = 2 * w + h, i = st - S0;   // K 32 st .. + 31: sub-blocks 2 st, 2 st + 1
+            const int sft = 4 * h, sb8 = 16 * h;     // their quants: shifts 4h, 4h + 2; scales: bytes 2h, 2h + 1
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t a0 = ((ql[p] >> sft) & 0x03030303u) * ((sl[p] >> sb8) & 15u);
+                const uint32_t a1 = ((qh[p] >> sft) & 0x03030303u) * ((sh[p] >> sb8) & 15u);
+                const uint32_t a2 = ((ql[p] >> (sft + 2)) & 0x03030303u) * ((sl[p] >> (sb8 + 8)) & 15u);
+                const uint32_t a3 = ((qh[p] >> (sft + 2)) & 0x03030303u) * ((sh[p] >> (sb8 + 8)) & 15u);
+                mma_u8s8_16832(chi[p], a0, a1, a2, a3, B[i][0], B[i][1]);
+                mma_u8u8_16832(clo[p], a0, a1, a2, a3, B[i][2], B[i][3]);
+            }
+        }
+    }
+    // minimum term: A = m of sub-blocks 2q, 2q+1 (k-slots 2q, 2q+1) and 2q+8, 2q+9
+    // (bytes 2 (q % 2), + 1 of sc|m words q / 2 and 2 + q / 2); a half keeps only
+    // its own sub-blocks
     auto mpair = [&](uint32_t w) {  // bytes 0, 1 of w -> their high nibbles as an f16 subnormal pair
         return ((w >> 4) & 0xFu) | ((w << 4) & 0xF0000u);
     };
     const int sh16 = 16 * (q & 1);
-    const uint32_t lA = (q < 2 ? ml.x : ml.y) >> sh16, lB = (q < 2 ? ml.z : ml.w) >> sh16;
-    const uint32_t hA = (q < 2 ? mh.x : mh.y) >> sh16, hB = (q < 2 ? mh.z : mh.w) >> sh16;
-    const uint32_t ma0 = HALF == 1 ? 0u : mpair(lA), ma1 = HALF == 1 ? 0u : mpair(hA);
-    const uint32_t ma2 = HALF == 0 ? 0u : mpair(lB), ma3 = HALF == 0 ? 0u : mpair(hB);
-    float tn[4];
-    mma_f16_16816_z(tn, ma0, ma1, ma2, ma3, bm[0], bm[1]);
-    mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[2], bm[3]);
-    const uint32_t dl = lds32(dd + (HALF < 0 ? scale_off(rg, sb) : rg * ddrow + 4 * sb));
-    const uint32_t dh = lds32(dd + (HALF < 0 ? scale_off(rh, sb) : rh * ddrow + 4 * sb));
-    // dmin: 2^24 undoes the subnormal encoding of m, 2^5 the sub-block-sum pre-scale
-    const float d0 = __half2float(__ushort_as_half((uint16_t)(dl & 0xFFFF)));
-    const float m0 = __half2float(__ushort_as_half((uint16_t)(dl >> 16))) * 536870912.0f;
-    const float d1 = __half2float(__ushort_as_half((uint16_t)(dh & 0xFFFF)));
-    const float m1 = __half2float(__ushort_as_half((uint16_t)(dh >> 16))) * 536870912.0f;
-    acc[0] = fmaf(-m0, tn[0], fmaf(d0, __int2float_rn(256 * chi[0] + clo[0]), acc[0]));
-    acc[1] = fmaf(-m0, tn[1], fmaf(d0, __int2float_rn(256 * chi[1] + clo[1]), acc[1]));
-    acc[2] = fmaf(-m1, tn[2], fmaf(d1, __int2float_rn(256 * chi[2] + clo[2]), acc[2]));
-    acc[3] = fmaf(-m1, tn[3], fmaf(d1, __int2float_rn(256 * chi[3] + clo[3]), acc[3]));
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        const uint32_t ma0 = HALF == 1 ? 0u : mpair(lds32(slp[p] + 4 * (q >> 1)) >> sh16);
+        const uint32_t ma1 = HALF == 1 ? 0u : mpair(lds32(shp[p] + 4 * (q >> 1)) >> sh16);
+        const uint32_t ma2 = HALF == 0 ? 0u : mpair(lds32(slp[p] + 8 + 4 * (q >> 1)) >> sh16);
+        const uint32_t ma3 = HALF == 0 ? 0u : mpair(lds32(shp[p] + 8 + 4 * (q >> 1)) >> sh16);
+        float tn[4];
+        mma_f16_16816_z(tn, ma0, ma1, ma2, ma3, bm[0], bm[1]);
+        mma_f16_16816(tn, ma0, ma1, ma2, ma3, bm[2], bm[3]);
+        const uint8_t *dd = P[p].dd;
+        const uint32_t dl = lds32(dd + (HALF < 0 ? scale_off(rg[p], sb) : rg[p] * ddrow + 4 * sb));
+        const uint32_t dh = lds32(dd + (HALF < 0 ? scale_off(rh[p], sb) : rh[p] * ddrow + 4 * sb));
+        // dmin: 2^24 undoes the subnormal encoding of m, 2^5 the sub-block-sum pre-scale
+        const float d0 = __half2float(__ushort_as_half((uint16_t)(dl & 0xFFFF)));
+        const float m0 = __half2float(__ushort_as_half((uint16_t)(dl >> 16))) * 536870912.0f;
+        const float d1 = __half2float(__ushort_as_half((uint16_t)(dh & 0xFFFF)));
+        const float m1 = __half2float(__ushort_as_half((uint16_t)(dh >> 16))) * 536870912.0f;
+        acc[p][0] = fmaf(-m0, tn[0], fmaf(d0, __int2float_rn(256 * chi[p][0] + clo[p][0]), acc[p][0]));
+        acc[p][1] = fmaf(-m0, tn[1], fmaf(d0, __int2float_rn(256 * chi[p][1] + clo[p][1]), acc[p][1]));
+        acc[p][2] = fmaf(-m1, tn[2], fmaf(d1, __int2float_rn(256 * chi[p][2] + clo[p][2]), acc[p][2]));
+        acc[p][3] = fmaf(-m1, tn[3], fmaf(d1, __int2float_rn(256 * chi[p][3] + clo[p][3]), acc[p][3]));
+    }
 }
 
 // B fragments of one super-block, or half of one (HALF as above), of an
@@ -869,18 +898,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             }
         } else if (Q2 && un.kind == kGrt) {
             const uint8_t *st = s.w[slot], *ss = s.s[slot];
-#pragma unroll
-            for (int m = 0; m < 2; ++m)
-                q2k_superblock<-1>(acc[m], st + 16384 * m, ss + 4096 * m, ss + kQDd + 1024 * m, 16, 64, 0, warp, g,
-                                   q, B, Bm);
+            const Q2Part P[2] = {{st, ss, ss + kQDd, 0}, {st + 16384, ss + 4096, ss + kQDd + 1024, 0}};
+            q2k_superblock2<-1>(acc, P, 16, 64, warp, g, q, B, Bm);
             release(slot);
         } else if (Q2 && un.kind == kDrt) {
             const uint8_t *st = s.w[slot], *ss = s.s[slot];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                if (warp & 1) q2k_superblock<1>(acc[t], st, ss, ss + kQDd, 32, 32, 16 * t, warp >> 1, g, q, B, Bm);
-                else q2k_superblock<0>(acc[t], st, ss, ss + kQDd, 32, 32, 16 * t, warp >> 1, g, q, B, Bm);
-            }
+            const Q2Part P[2] = {{st, ss, ss + kQDd, 0}, {st, ss, ss + kQDd, 16}};
+            if (warp & 1) q2k_superblock2<1>(acc, P, 32, 32, warp >> 1, g, q, B, Bm);
+            else q2k_superblock2<0>(acc, P, 32, 32, warp >> 1, g, q, B, Bm);
             release(slot);
         } else if (un.kind == kGrt) {
             // two stages of K 2048: W1 rows at +0, W3 rows at +16384; E8M0 scale

@@ -24,10 +24,9 @@
 //  - the epilogue thread is a weight row (TMEM lane), its columns tokens:
 //    h = bf16(silu(g) u) goes to h [S][d_ff] (K-major for the down GEMM), the
 //    down rows to out_rows [S][d_model] in fp32.
-// One persistent CTA per SM: a TMA warp, an MMA warp, twelve decoder warps
-// (three per TMEM lane quarter, taking the stages in turn) and four epilogue
-// warps; an 8-stage shared-memory ring (token rows + codes) ahead of a 4-stage
-// tensor-memory ring (decoded A); every wait is bounded.
+// One persistent CTA per SM: a TMA warp, an MMA warp, four decoder warps and
+// eight epilogue warps; an 8-stage shared-memory ring (token rows + codes)
+// ahead of a 4-stage tensor-memory ring (decoded A); every wait is bounded.
 #include <string.h>
 
 #include <atomic>
@@ -44,8 +43,10 @@ namespace {
 
 constexpr int k16Sm = 8;          // shared-memory stages: token rows and weight codes
 constexpr int k16Ta = 4;          // tensor-memory stages: decoded weights
-constexpr int k16Dec = 3;         // decoder warps per TMEM lane quarter (they take turns by stage)
-constexpr int k16Threads = 576;   // warp 0 TMA, 1 MMA, 2..13 decoders, 14..17 epilogue
+constexpr int k16Dec = 1;         // decoder warps per TMEM lane quarter (they would take turns by stage;
+                                  // three measured 5% slower: the MMAs, not the decoders, set the pace)
+constexpr int k16Epi = 2;         // epilogue warps per TMEM lane quarter (each a share of the tokens)
+constexpr int k16Threads = 32 * (2 + 4 * k16Dec + 4 * k16Epi);  // warp 0 TMA, 1 MMA, decoders, epilogue
 constexpr int k16Tile = 128;      // weight rows (M) and tokens (N) per tile
 constexpr int k16Kst = 64;        // K per stage (one 128-byte row of bf16)
 constexpr int k16MaxE = 1024;
@@ -167,7 +168,7 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
             mbar_init(&s.aempty[i], 1);
         }
         mbar_init(&s.acc_full, 1);
-        mbar_init(&s.acc_empty, 4);
+        mbar_init(&s.acc_empty, 4 * k16Epi);
         mbar_init(&s.mma_done, 1);
         s.abort = 0;
         fence_mbar_init();
@@ -287,8 +288,9 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
     } else {
         // ------------------------------ epilogue ------------------------------
         // TMEM lane = weight row (this warp: quarter q), columns = the tile's
-        // tokens, in four chunks of 32.
-        const int q = warp & 3, r = 32 * q + lane;
+        // tokens in chunks of 32; epilogue warp e of a quarter takes chunks
+        // e, e + k16Epi, ...
+        const int q = warp & 3, e = (warp - 2 - 4 * k16Dec) >> 2, r = 32 * q + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         int lw = 0;
         for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++lw) {
@@ -302,7 +304,7 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
             tc_fence_after();
             const int col = wk.f * k16Tile + r;  // this thread's output feature (gate/up: row of h)
 #pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = e; cc < 4; cc += k16Epi) {
                 const int t0 = 32 * cc;            // first token of this chunk
                 if (t0 >= wk.nvalid) break;      // warp-uniform
                 uint32_t g[32], u[32];
