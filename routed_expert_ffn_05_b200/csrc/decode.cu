@@ -72,7 +72,10 @@ constexpr int kMaxSeg = 256;              // active experts of a decode batch: m
 // column); the consumers' fragment stores conflict at most 2-way.
 constexpr int kRedM = 144, kRedR = 9;
 constexpr int kD = 4096, kF = 2048;       // the dims this tiling is written for
-constexpr int kGuTiles = kF / 16;         // gate/up tiles per routed expert
+// A routed gate/up unit: 32 rows of W1 and W3 over all K for MXFP4 (two
+// 16-row halves of two stages each, one hand-off), 16 rows (one stage) for Q2_K.
+template <int WF> constexpr int gu_rows() { return WF == MOE_W_Q2K ? 16 : 32; }
+template <int WF> constexpr int gu_tiles() { return kF / gu_rows<WF>(); }  // units per routed expert
 // A routed down unit: 64 W2 rows over all K (two stages of 32 rows) for
 // MXFP4, 32 rows (one stage) for Q2_K; its partial tiles are 16 rows each.
 // (A 64-row Q2_K unit in one stage, with three stages to make room for its
@@ -177,16 +180,16 @@ __device__ __forceinline__ int active_experts(const int32_t *offsets, int E, int
 // kernels run. The shared down units sit between the two routed phases, where
 // they need no wait (every shared gate/up tile is long done) and cover the
 // tail of the routed gate/up phase. A routed gate/up unit is 16 rows of W1 and
-// W3 over all K: two stages of MXFP4 codes, or one stage of Q2_K quants (half
-// the bytes).
-template <int WF> constexpr int gu_stages() { return WF == MOE_W_Q2K ? 1 : 2; }
+// W3 over all K: four stages of MXFP4 codes (two per 16 rows), or one stage
+// of Q2_K quants (16 rows, half the bytes per row).
+template <int WF> constexpr int gu_stages() { return WF == MOE_W_Q2K ? 1 : 4; }
 
 template <int WF>
 __device__ __forceinline__ Unit unit_of(int u, int usg, int n_seg, int usd) {
     if (u < usg) return Unit{kGsh, -1, u, 8};
     int r = u - usg;
-    if (r < n_seg * kGuTiles) return Unit{kGrt, r / kGuTiles, r % kGuTiles, gu_stages<WF>()};
-    r -= n_seg * kGuTiles;
+    if (r < n_seg * gu_tiles<WF>()) return Unit{kGrt, r / gu_tiles<WF>(), r % gu_tiles<WF>(), gu_stages<WF>()};
+    r -= n_seg * gu_tiles<WF>();
     if (r < usd) return Unit{kDsh, -1, r, 2};
     r -= usd;
     return Unit{kDrt, r / dn_tiles<WF>(), r % dn_tiles<WF>(), dn_stages<WF>()};
@@ -484,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         int gi = 0;
         auto issue = [&](int u, const Unit &un) {
             int row0 = 0;
-            if (un.kind == kGrt) row0 = s.seg_e[un.seg] * kF + 16 * un.tile;
+            if (un.kind == kGrt) row0 = s.seg_e[un.seg] * kF + gu_rows<WF>() * un.tile;
             if (un.kind == kDrt) row0 = s.seg_e[un.seg] * kD + dn_rows<WF>() * un.tile;
             for (int c = 0; c < un.nst && !s.abort; ++c, ++gi) {
                 const int slot = gi % kStages;
@@ -507,12 +510,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                             tma_load_3d(sm + 4096, &a.m3s, 0, row0, 0, bar);
                             tma_load_2d(sm + kQDd, &a.m1d, 0, row0, bar);
                             tma_load_2d(sm + kQDd + 1024, &a.m3d, 0, row0, bar);
-                        } else {
+                        } else {  // stage c: rows row0 + 16 (c / 2) .. + 15, K half c % 2
+                            const int rr = row0 + 16 * (c >> 1), kh = c & 1;
                             arm(s, slot, u, un, 2 * 16384 + 2 * 1024);
-                            tma_load_3d(w, &a.m1c, 0, row0, 8 * c, bar);
-                            tma_load_3d(w + 16384, &a.m3c, 0, row0, 8 * c, bar);
-                            tma_load_2d(sm, &a.m1s, 64 * c, row0, bar);
-                            tma_load_2d(sm + 1024, &a.m3s, 64 * c, row0, bar);
+                            tma_load_3d(w, &a.m1c, 0, rr, 8 * kh, bar);
+                            tma_load_3d(w + 16384, &a.m3c, 0, rr, 8 * kh, bar);
+                            tma_load_2d(sm, &a.m1s, 64 * kh, rr, bar);
+                            tma_load_2d(sm + 1024, &a.m3s, 64 * kh, rr, bar);
                         }
                         break;
                     case kDsh:
@@ -560,12 +564,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         if (lane != 0) return;
         s.n_seg = n;
         const int G = (int)gridDim.x;
-        const int gu_end = usg + n * kGuTiles;
+        const int gu_end = usg + n * gu_tiles<WF>();
         // Routed gate/up tickets: G chunks of cb units that hold three quarters
         // of the work (one per CTA when all run at once), then chunks of kGrab
         // units, which even out CTAs that started late or ran slow.
         constexpr int kGrab = 2;
-        const int R = n * kGuTiles;
+        const int R = n * gu_tiles<WF>();
         const int cb = (R - R / 4) / G;
         const int nb = cb >= kGrab ? G : 0;
         const int t_small = usg + nb, t_dn = t_small + (R - nb * cb + kGrab - 1) / kGrab;
@@ -693,7 +697,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             };
             const int row = lane & 15;
             if (un.kind == kGsh || un.kind == kGrt) {
-                // lanes 0..15: gate of rows 0..15, lanes 16..31: up
+                // lanes 0..15: gate of rows 0..15, lanes 16..31: up (a routed
+                // unit: per 16-row half p, tiles 2p (gate) and 2p + 1 (up))
                 const int col = 16 * un.tile + row;
                 if (un.kind == kGsh) {
                     for (int c = 0; c < a.T; ++c) {
@@ -708,14 +713,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     for (int i = 0; i < cnt; ++i) {  // the expert's rows; column = the row's token
                         const int tok = s.ep_tok[un.seg][i];
                         const float xs = s.ep_xs[tok];
-                        const float v = colsum(tok);
-                        const float up = __shfl_down_sync(0xffffffffu, v, 16);
-                        uint32_t hb = 0;
-                        if (lane < 16) {
-                            hb = f32_to_bf16_rne(silu_f32(v * xs) * (up * xs));
-                            a.h[(int64_t)(rbase + i) * kF + col] = (uint16_t)hb;
+                        uint32_t hmx = 0;
+#pragma unroll
+                        for (int p = 0; p < gu_rows<WF>() / 16; ++p) {
+                            const float v = colsum(tok, p);
+                            const float up = __shfl_down_sync(0xffffffffu, v, 16);
+                            if (lane < 16) {
+                                const uint32_t hb = f32_to_bf16_rne(silu_f32(v * xs) * (up * xs));
+                                a.h[(int64_t)(rbase + i) * kF + gu_rows<WF>() * un.tile + 16 * p + row] = (uint16_t)hb;
+                                hmx = max(hmx, (hb & 0x7FFFu) << 16);
+                            }
                         }
-                        const uint32_t mx = warp_max_bits((hb & 0x7FFFu) << 16);
+                        const uint32_t mx = warp_max_bits(hmx);
                         if (lane == 0) atomicMax(&a.hmax[rbase + i], mx);
                     }
                     if (un.seg != pseg) {  // a new expert: the previous one's count goes out
@@ -834,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     flushed = true;
                 }
                 const bool ok = un.kind == kDsh ? wait_count(sh_done, (uint32_t)usg, lane, &s.abort)
-                                                : wait_count(seg_done + un.seg, (uint32_t)kGuTiles, lane, &s.abort);
+                                                : wait_count(seg_done + un.seg, (uint32_t)gu_tiles<WF>(), lane, &s.abort);
                 if (!ok) { fail(a, s); return; }
             }
             if (Q2 && un.kind == kGrt) {  // x: super-block `warp` of K
@@ -908,25 +917,39 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             else q2k_superblock2<0>(acc, P, 32, 32, warp >> 1, g, q, B, Bm);
             release(slot);
         } else if (un.kind == kGrt) {
-            // two stages of K 2048: W1 rows at +0, W3 rows at +16384; E8M0 scale
-            // word w of rows g, g + 8 (W3's 1024 bytes further)
+            // two 16-row halves of two stages of K 2048 each: W1 rows at +0, W3
+            // rows at +16384; E8M0 scale word w of rows g, g + 8 (W3's 1024
+            // bytes further). The partial tiles go out per half (tiles 2h: gate,
+            // 2h + 1: up), so the buffer is claimed first.
+            if (!mbar_wait(&s.rempty[ru & 1], ((ru >> 1) & 1) ^ 1, &s.abort)) { fail(a, s); return; }
+            float *red = s.red[ru & 1][warp];
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                if (h > 0) {
+                    if (!next_stage()) { fail(a, s); return; }
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                if (c > 0 && !next_stage()) { fail(a, s); return; }
-                const uint32_t cw = w_base + (uint32_t)slot * kStageW;
-                const uint32_t cs = w_base + kScaleBase + (uint32_t)slot * kStageS + sc_lo;
-                uint32_t sw[2][2];
-                sw[0][0] = lds32_at<0>(cs);
-                sw[0][1] = lds32_at<512>(cs);
-                sw[1][0] = lds32_at<1024>(cs);
-                sw[1][1] = lds32_at<1536>(cs);
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint32_t ad = cw + code_off(code_gu, jj);
-                    mxfp4_block<0>(acc[0], ad, sw[0][0], sw[0][1], jj, B[4 * c + jj]);
-                    mxfp4_block<16384>(acc[1], ad, sw[1][0], sw[1][1], jj, B[4 * c + jj]);
+                    for (int m = 0; m < 2; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
                 }
-                release(slot);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    if (c > 0 && !next_stage()) { fail(a, s); return; }
+                    const uint32_t cw = w_base + (uint32_t)slot * kStageW;
+                    const uint32_t cs = w_base + kScaleBase + (uint32_t)slot * kStageS + sc_lo;
+                    uint32_t sw[2][2];
+                    sw[0][0] = lds32_at<0>(cs);
+                    sw[0][1] = lds32_at<512>(cs);
+                    sw[1][0] = lds32_at<1024>(cs);
+                    sw[1][1] = lds32_at<1536>(cs);
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const uint32_t ad = cw + code_off(code_gu, jj);
+                        mxfp4_block<0>(acc[0], ad, sw[0][0], sw[0][1], jj, B[4 * c + jj]);
+                        mxfp4_block<16384>(acc[1], ad, sw[1][0], sw[1][1], jj, B[4 * c + jj]);
+                    }
+                    release(slot);
+                }
+                put_partial(red + 2 * kRedM * h, g, q, acc[0]);
+                put_partial(red + (2 * h + 1) * kRedM, g, q, acc[1]);
             }
         } else if (un.kind == kDsh) {
 #pragma unroll
@@ -968,10 +991,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                 put_partial(red + (2 * c + 1) * kRedM, g, q, acc[1]);
             }
         }
-        // hand the unit (or tile) to the epilogue warp (MXFP4 down units have
-        // put their tiles in place already)
+        // hand the unit (or tile) to the epilogue warp (routed MXFP4 units and
+        // Q2_K down units have put their tiles in place already)
         const int rb = ru & 1;
-        if (Q2 || un.kind != kDrt) {
+        if (un.kind == kGsh || un.kind == kDsh || (Q2 && un.kind == kGrt) || (Q2 && un.kind == kDrt)) {
             if (!mbar_wait(&s.rempty[rb], ((ru >> 1) & 1) ^ 1, &s.abort)) { fail(a, s); return; }
             // bf16 and Q2_K tiles read rows sigma(g)
             const int rg = (Q2 || un.kind == kGsh || un.kind == kDsh) ? sigma(g) : g;
