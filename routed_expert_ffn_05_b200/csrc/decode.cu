@@ -574,15 +574,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         const int nb = cb >= kGrab ? G : 0;
         const int t_small = usg + nb, t_dn = t_small + (R - nb * cb + kGrab - 1) / kGrab;
         // Down tickets: G contiguous ranges of equal cost over the shared and
-        // routed down units (shared tiles cost 2 stages, routed ones dn_stages),
-        // so a CTA changes expert, and reloads its h fragments, once or twice.
-        constexpr int kDst = dn_stages<WF>();
+        // routed down units (shared tiles cost 2 stages, routed ones dn_stages)
+        // that hold seven eighths of the work, so a CTA changes expert, and
+        // reloads its h fragments, once or twice; then chunks of kGrabD units,
+        // which even out CTAs that reached the down phase late.
+        constexpr int kDst = dn_stages<WF>(), kGrabD = 2;
         const long long cost = 2ll * usd + (long long)n * dn_tiles<WF>() * kDst;
+        const long long cost_big = cost - cost / 8;
         auto first = [&](long long cst) {
             return gu_end + (cst <= 2ll * usd ? (int)((cst + 1) / 2)
                                               : usd + (int)((cst - 2ll * usd + kDst - 1) / kDst));
         };
-        const int t_end = t_dn + G;
+        const int dn_end = gu_end + usd + n * dn_tiles<WF>();
+        const int u_small = first(cost_big);
+        const int t_dsmall = t_dn + G;
+        const int t_end = t_dsmall + (dn_end - u_small + kGrabD - 1) / kGrabD;
         while (t < t_end && !s.abort) {
             int u0, u1;
             if (t < usg) {
@@ -594,9 +600,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             } else if (t < t_dn) {
                 u0 = usg + nb * cb + (t - t_small) * kGrab;
                 u1 = min(u0 + kGrab, gu_end);
+            } else if (t < t_dsmall) {
+                u0 = first(cost_big * (t - t_dn) / G);
+                u1 = first(cost_big * (t - t_dn + 1) / G);
             } else {
-                u0 = first(cost * (t - t_dn) / G);
-                u1 = first(cost * (t - t_dn + 1) / G);
+                u0 = u_small + (t - t_dsmall) * kGrabD;
+                u1 = min(u0 + kGrabD, dn_end);
             }
             // The next chunk is claimed while this chunk's last unit is issued
             // (the ring keeps the consumers a few stages behind), not earlier:
