@@ -34,3 +34,50 @@ def test_reference_arm_prints_the_contract_line():
                         "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] and d["config"]["T"] == 4
     assert d["vs_baseline"] is None and d["data"] == "synthetic"
+
+
+def test_peaks_burst_and_sustained():
+    """The roofline denominators come from the measured-peaks file: the burst
+    bf16 figure by default, the sustained one for a run that met the power cap."""
+    import bench
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    hbm, bf16, src = bench.peaks()
+    hbm_s, bf16_s, src_s = bench.peaks(sustained=True)
+    if os.path.exists(path):
+        with open(path) as f:
+            j = json.load(f)
+        assert (hbm, bf16, src) == (j["hbm_gbs"], j["bf16_tflops"], "measured")
+        assert hbm_s == j["hbm_gbs"] and bf16_s == j["bf16_tflops_sustained"] and src_s == "measured sustained"
+        assert bf16_s < bf16
+    else:
+        assert src == "fallback" and src_s == "fallback sustained"
+
+
+def test_captured_traffic_only_for_its_workload_and_sources(monkeypatch):
+    """A recorded DRAM figure is reported for its own workload while the kernel
+    sources hash to the recorded value, and never for another workload or after
+    a source change."""
+    import bench
+    import synth
+    from dataclasses import replace
+    rec = bench.TRAFFIC[0]
+    cfg = synth.CONFIGS[rec["config"]]
+    T = rec["T"]
+    live = bench.sources_sha256(rec["sources"])
+    monkeypatch.setitem(rec, "sources_sha256", live)
+    assert bench.captured_traffic(replace(cfg, E=rec["E"]), T) == (rec["dram_bytes"], rec["kernels"])
+    assert bench.captured_traffic(replace(cfg, E=rec["E"]), T + 1) == (None, None)     # other T
+    assert bench.captured_traffic(replace(cfg, E=rec["E"] // 4), T) == (None, None)    # other E
+    monkeypatch.setitem(rec, "sources_sha256", "0" * 64)                               # sources changed
+    assert bench.captured_traffic(replace(cfg, E=rec["E"]), T) == (None, None)
+
+
+def test_oracle_thread_count_is_settable():
+    """The single-threaded CPU baseline runs the same oracle on one thread."""
+    import oracle
+    n = oracle.num_threads()
+    try:
+        assert oracle.set_num_threads(1) == 1 and oracle.num_threads() == 1
+    finally:
+        oracle.set_num_threads(n)
+    assert oracle.num_threads() == n
