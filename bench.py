@@ -165,7 +165,7 @@ def algorithmic_ffn_bytes(cfg, n_experts_touched):
 #  - decode T=8: one decode_ffn_kernel launch on batch 0 (58 experts touched);
 #    command and figures in profiles/decode_ffn_kernel_traffic_decode_T8.md.
 #  - prefill T=4096 (w4a8): the gate/up and the down tc_ffn_kernel launches of
-#    one layer call (batch 2), summed: 1,675.7 + 1,053.1 MB; command and figures
+#    one layer call (batch 2), summed: 1,663.6 + 1,052.7 MB; command and figures
 #    in profiles/tc_ffn_kernel_traffic_prefill_T4096.md.
 _DECODE_SOURCES = ["routed_expert_ffn_05_b200/csrc/decode.cu", "routed_expert_ffn_05_b200/csrc/common.cuh",
                    "routed_expert_ffn_05_b200/csrc/kernels.h", "routed_expert_ffn_05_b200/csrc/ptx.cuh",
@@ -177,12 +177,12 @@ _PREFILL_SOURCES = ["routed_expert_ffn_05_b200/csrc/prefill.cu", "routed_expert_
                     "routed_expert_ffn_05_b200/csrc/tma.cu", "routed_expert_ffn_05_b200/csrc/layout.h",
                     "include/moe.h"]
 TRAFFIC = [
-    {"config": "decode", "T": 8, "E": 256, "act": "bf16", "dram_bytes": 830_619_648,
+    {"config": "decode", "T": 8, "E": 256, "act": "bf16", "dram_bytes": 830_582_272,
      "kernels": "decode_ffn_kernel<MXFP4>", "sources": _DECODE_SOURCES,
-     "sources_sha256": "ccd317a67845afeca0b3840c936f65951827712eb6daf8935501aeb174f50361"},
-    {"config": "prefill", "T": 4096, "E": 256, "act": "mxfp8", "dram_bytes": 2_728_790_784,
+     "sources_sha256": "b6e18134afe13e6fff6d6e07c10d2a4ffe9d43af05a35da5646a16db24a45060"},
+    {"config": "prefill", "T": 4096, "E": 256, "act": "mxfp8", "dram_bytes": 2_716_298_752,
      "kernels": "tc_ffn_kernel gate/up + down", "sources": _PREFILL_SOURCES,
-     "sources_sha256": "472b95716d34353f4061ce0dba9604279a0dfc4fcb14076159801c7c1024be09"},
+     "sources_sha256": "c862a96bbd813162f84bb2f9ee89fa05f70c4b0d79dbebc772f67d10a14883fc"},
 ]
 
 
