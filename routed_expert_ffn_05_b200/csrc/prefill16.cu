@@ -70,7 +70,7 @@ struct T16Smem {
     uint8_t b[k16Sm][k16Tile * 128];      // token rows: 128 rows x K 64 (bf16)
     uint8_t wc[k16Sm][2][k16Tile * 32];   // weight codes: 128 rows x K 64 (E2M1) per matrix
     uint8_t wsf[k16Sm][2][512];           // the scale atom holding the stage's K 64 per matrix
-    uint64_t full[k16Sm], sempty[k16Sm], a_full[k16Ta], aempty[k16Ta], acc_full, acc_empty, mma_done;
+    uint64_t full[k16Sm], sempty[k16Sm], a_full[k16Ta], aempty[k16Ta], acc_full[2], acc_empty[2], mma_done;
     uint32_t tmem_base;
     volatile int abort;
     int ustart[k16MaxE + 1];
@@ -154,7 +154,10 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool GU = MODE == kGU16;
     constexpr int kMats = GU ? 2 : 1;          // weight matrices per item: W1 and W3, or W2
-    constexpr uint32_t kAcc = GU ? 256u : 128u;  // accumulator columns: g | u, or o
+    // accumulator columns: gate/up one buffer of g | u (256); down two buffers
+    // of o (128 each), so the epilogue of one item overlaps the next item's MMAs
+    constexpr int kNb = GU ? 1 : 2;
+    constexpr uint32_t kAcc = 256u;              // A stages start here
     constexpr uint32_t kAStage = 32u * kMats;    // A columns per stage
     const int ft = a.Nw / k16Tile, kt_n = a.K / k16Kst;
 
@@ -167,8 +170,10 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
             mbar_init(&s.a_full[i], 4);  // one arrival per decoder warp
             mbar_init(&s.aempty[i], 1);
         }
-        mbar_init(&s.acc_full, 1);
-        mbar_init(&s.acc_empty, 4 * k16Epi);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.acc_full[i], 1);
+            mbar_init(&s.acc_empty[i], 4 * k16Epi);
+        }
         mbar_init(&s.mma_done, 1);
         s.abort = 0;
         fence_mbar_init();
@@ -216,8 +221,10 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
             constexpr uint32_t idesc = idesc_bf16(k16Tile, k16Tile);
             int it = 0, lw = 0;
             for (int w = blockIdx.x; w < n_work && !s.abort; w += gridDim.x, ++lw) {
-                if (!mbar_wait(&s.acc_empty, (lw & 1) ^ 1, &s.abort)) { t16_fail(a, s); break; }
+                const int ab = lw % kNb;  // accumulator buffer of this item
+                if (!mbar_wait(&s.acc_empty[ab], ((lw / kNb) & 1) ^ 1, &s.abort)) { t16_fail(a, s); break; }
                 tc_fence_after();
+                const uint32_t dacc = tmem + 128u * (uint32_t)ab;
                 bool ok = true;
                 for (int kt = 0; kt < kt_n; ++kt, ++it) {
                     const int slot = it % k16Sm, ta = it % k16Ta;
@@ -232,14 +239,14 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {  // K = 16: 8 TMEM columns of A, 32 bytes of every B row
                         const uint32_t acc = (kt | ks) != 0;
-                        tc_mma_bf16_ts(tmem, a0 + 8 * ks, db + 2 * ks, idesc, acc);
+                        tc_mma_bf16_ts(dacc, a0 + 8 * ks, db + 2 * ks, idesc, acc);
                         if (GU) tc_mma_bf16_ts(tmem + 128, a0 + 32 + 8 * ks, db + 2 * ks, idesc, acc);
                     }
                     tc_commit(&s.sempty[slot]);  // the shared stage and
                     tc_commit(&s.aempty[ta]);    // the A columns are free once these finish
                 }
                 if (!ok) { t16_fail(a, s); break; }
-                tc_commit(&s.acc_full);
+                tc_commit(&s.acc_full[ab]);
             }
             tc_commit(&s.mma_done);
             mbar_wait(&s.mma_done, 0);
@@ -296,21 +303,32 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
         for (int w = blockIdx.x; w < n_work; w += gridDim.x, ++lw) {
             if (__shfl_sync(0xffffffffu, s.abort, 0)) break;
             const Work16 wk = work16_of(w, ft, s.ustart, a.E, a.offsets);
-            const bool ok = mbar_wait(&s.acc_full, lw & 1, &s.abort);
+            const int ab = lw % kNb;
+            const bool ok = mbar_wait(&s.acc_full[ab], (lw / kNb) & 1, &s.abort);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) t16_fail(a, s);
                 break;
             }
             tc_fence_after();
             const int col = wk.f * k16Tile + r;  // this thread's output feature (gate/up: row of h)
+            // the accumulator goes back as soon as this warp's last chunk is in registers
+            int last = -1;
+            for (int cc = e; cc < 4; cc += k16Epi)
+                if (32 * cc < wk.nvalid) last = cc;
+            auto release = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.acc_empty[ab]);
+            };
+            if (last < 0) release();
 #pragma unroll 1
-            for (int cc = e; cc < 4; cc += k16Epi) {
+            for (int cc = e; cc <= last; cc += k16Epi) {
                 const int t0 = 32 * cc;            // first token of this chunk
-                if (t0 >= wk.nvalid) break;      // warp-uniform
                 uint32_t g[32], u[32];
-                tmem_ld32(lane_base + t0, g);
+                tmem_ld32(lane_base + 128u * (uint32_t)ab + t0, g);
                 if (GU) tmem_ld32(lane_base + 128 + t0, u);
                 tmem_wait_ld();
+                if (cc == last) release();
                 const int nv = min(32, wk.nvalid - t0);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -320,9 +338,6 @@ __global__ void __launch_bounds__(k16Threads, 1) tc16_ffn_kernel(const __grid_co
                     else a.out[o] = __uint_as_float(g[i]);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.acc_empty);
         }
     }
     tc_fence_before();
