@@ -49,7 +49,7 @@ def cfg_of(name, T=None):
 
 
 LAYER_CASES = [("tiny", None), ("decode", 1), ("decode", 2), ("decode", 4), ("decode", 8),
-               ("q2k", 1), ("q2k", 8), ("q2k", 16), ("prefill", None), ("hash", None)]
+               ("q2k", 1), ("q2k", 8), ("q2k", 16), ("prefill", 9), ("prefill", None), ("hash", None)]
 _cases = {}
 
 

@@ -37,6 +37,8 @@ def rel_err(got, ref):
 CASES = [
     ("small-ragged", synth.LayerConfig("w4a16", T=300, d=256, F=512, E=8, k=3)),
     ("small-one-token", synth.LayerConfig("w4a16", T=1, d=512, F=256, E=4, k=2)),
+    ("decode-dims-T9", replace(synth.CONFIGS["decode"], T=9)),     # one token past the decode kernel
+    ("decode-dims-T31", replace(synth.CONFIGS["decode"], T=31)),    # below the tensor-core router
     ("decode-dims-T64", replace(synth.CONFIGS["decode"], T=64)),
     ("prefill-dims", replace(synth.CONFIGS["prefill"], T=384, act="bf16")),
 ]
