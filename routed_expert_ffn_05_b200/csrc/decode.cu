@@ -84,7 +84,14 @@ template <int WF> constexpr int dn_rows() { return WF == MOE_W_Q2K ? 32 : 64; }
 template <int WF> constexpr int dn_parts() { return dn_rows<WF>() / 32; }
 template <int WF> constexpr int dn_stages() { return dn_parts<WF>(); }
 template <int WF> constexpr int dn_tiles() { return kD / dn_rows<WF>(); }
-template <int WF> constexpr int red_w() { return dn_rows<WF>() / 16 * kRedM; }  // floats per warp
+// A consumer warp's partial-tile buffer holds one unit's 16-row tiles: a
+// routed gate/up unit's (two matrices per 16 rows) or a down unit's, whichever
+// is more (the shared expert's units need two). Floats per warp.
+template <int WF> constexpr int red_tiles() {
+    return dn_rows<WF>() / 16 > 2 * gu_rows<WF>() / 16 ? dn_rows<WF>() / 16 : 2 * gu_rows<WF>() / 16;
+}
+template <int WF> constexpr int red_w() { return red_tiles<WF>() * kRedM; }
+static_assert(red_tiles<MOE_W_MXFP4>() >= 2 && red_tiles<MOE_W_Q2K>() >= 2, "partial tiles");
 constexpr int kDshTiles = kD / 16;        // shared-expert down tiles
 
 // Work kinds: shared gate/up (bf16, 8 stages of K 512), routed gate/up (MXFP4,
