@@ -177,9 +177,9 @@ _PREFILL_SOURCES = ["routed_expert_ffn_05_b200/csrc/prefill.cu", "routed_expert_
                     "routed_expert_ffn_05_b200/csrc/tma.cu", "routed_expert_ffn_05_b200/csrc/layout.h",
                     "include/moe.h"]
 TRAFFIC = [
-    {"config": "decode", "T": 8, "E": 256, "act": "bf16", "dram_bytes": 830_543_360,
+    {"config": "decode", "T": 8, "E": 256, "act": "bf16", "dram_bytes": 830_646_272,
      "kernels": "decode_ffn_kernel<MXFP4>", "sources": _DECODE_SOURCES,
-     "sources_sha256": "12d80d1215da344e04df22aecd98c4fae75dc3d9134961b196042158148fc74f"},
+     "sources_sha256": "d272df0938e8275eb145116ac62269d8c428e775d927e12955e80fd333971d6b"},
     {"config": "prefill", "T": 4096, "E": 256, "act": "mxfp8", "dram_bytes": 2_716_298_752,
      "kernels": "tc_ffn_kernel gate/up + down", "sources": _PREFILL_SOURCES,
      "sources_sha256": "c862a96bbd813162f84bb2f9ee89fa05f70c4b0d79dbebc772f67d10a14883fc"},

@@ -9,9 +9,10 @@
 //  - one CTA per SM with three roles: a producer thread moves weight tiles
 //    HBM -> shared memory with TMA (16-32 KB boxes, 128-byte swizzled; the
 //    E8M0 scale boxes 64-byte swizzled) through four mbarrier stages; sixteen
-//    consumer warps split K and run mma.sync m16n8k16 (16 weight rows x 8
-//    tokens, fp32 accumulate); an epilogue warp sums the consumers' partial
-//    tiles (double-buffered) and writes the outputs;
+//    consumer warps split K and run mma.sync (16 weight rows x 8 tokens:
+//    m16n8k16 f16 with fp32 accumulation for MXFP4, m16n8k32 integer for the
+//    Q2_K main term); an epilogue warp sums the consumers' partial tiles
+//    (double-buffered) and writes the outputs;
 //  - the work is numbered in units (a unit: one or more stages the consumers
 //    run back to back, then one hand-off to the epilogue): shared gate/up
 //    (streamed while routing finishes), routed gate/up, then down units; a
@@ -19,7 +20,8 @@
 //    tiles. CTAs claim the work in chunks from one ticket counter, in unit
 //    order: shared gate/up units one at a time, routed gate/up as one large
 //    chunk per CTA's worth of three quarters of it and then pairs, down units
-//    as contiguous cost-balanced ranges. Every unit a down unit waits for was
+//    as contiguous cost-balanced ranges over seven eighths of them and then
+//    pairs. Every unit a down unit waits for was
 //    claimed earlier by a CTA that is running and finishes its earlier claims
 //    first, so the kernel needs no co-residency of its CTAs (other work may
 //    hold some SMs, or a second layer may run on another stream);
