@@ -256,6 +256,31 @@ def test_two_decode_layers_on_two_streams():
     assert_rel(host(yb), ref_b, TOL["bf16"], "stream 2")
 
 
+@pytest.mark.parametrize("name", ["decode", "q2k"])
+def test_decode_wide_range_activations(name):
+    """Activations spanning twelve binades within a token (N(0, 1) times
+    2^u, u uniform in [-10, 2]): the decode kernel's per-token power-of-two
+    prescale (f16 for MXFP4; the 16-bit integer split for the Q2_K main term,
+    exact within 2^7 of the token's largest element) keeps the layer within
+    the w4a16 bound of the fp64 oracle."""
+    from harness import host_weights
+    cfg = synth.CONFIGS[name].with_T(2)
+    rng = np.random.default_rng(77)
+    xf = (rng.standard_normal((cfg.T, cfg.d)) * np.exp2(rng.uniform(-10, 2, (cfg.T, cfg.d)))).astype(np.float32)
+    xw = (xf.view(np.uint32) >> 16).astype(np.uint16)            # bf16 by truncation: exact bits, any rounding will do
+    idx, _ = oracle.topk_softmax(oracle.router_logits(xw, synth.make_router(cfg), synth.make_bias(cfg)), cfg.k)
+    host_weights(cfg).ensure(np.unique(idx))   # the experts this batch routes to, before the device copy is packed
+    c = Case(cfg)
+    ora = c.hw.oracle_layer(cfg, c.wr, c.bias, c.shared)
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.float32, device=DEV)
+    M.moe_layer(c.dims, c.weights, dev(xw), None, y, c.ws)
+    assert M.moe_get_device_error() == 0
+    toks = np.arange(cfg.T, dtype=np.int32)
+    got_idx, _, ref = oracle.layer_tokens(ora, xw, toks)
+    np.testing.assert_array_equal(got_idx, idx)
+    assert_rel(host(y), ref, TOL["bf16"], f"{name} wide-range x")
+
+
 # ---- the batch router on the tensor cores ------------------------------------------
 
 def _router_bound(x, wnorm, approx, bias, d):
